@@ -1,0 +1,566 @@
+// tq_api.cu -- the C ABI of libtq (see include/tq.h): argument checks, kernel
+// selection and launches.  No allocation, no synchronisation.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/tq.h"
+#include "tq_common.cuh"
+#include "tq_decode.cuh"
+#include "tq_dmma.cuh"
+#include "tq_rht.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return TQ_ERR_CUDA;
+}
+
+#define TQ_CUDA(call)                           \
+  do {                                          \
+    cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+int g_arch_ok[kMaxDevices];  // 0 unknown, 1 ok, 2 bad
+int g_num_sms[kMaxDevices];
+
+// Current device must be compute capability 10.0 (B200, sm_100a).
+int check_arch(int* num_sms) {
+  int dev = 0;
+  TQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return TQ_ERR_ARCH;
+  if (g_arch_ok[dev] == 0) {
+    int major = 0, minor = 0, sms = 0;
+    TQ_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    TQ_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    TQ_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    g_num_sms[dev] = sms;
+    g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  if (g_arch_ok[dev] != 1) return TQ_ERR_ARCH;
+  if (num_sms) *num_sms = g_num_sms[dev];
+  return TQ_OK;
+}
+
+bool k_ok(int32_t k) { return k > 0 && k % 512 == 0; }
+
+int check_weight(const tq_weight_t* w) {
+  if (!w) return TQ_ERR_NULL;
+  if (w->n < 1 || !k_ok(w->k)) return TQ_ERR_SHAPE;
+  if (!w->codes_d || !w->scales_d || !w->codebook_d) return TQ_ERR_NULL;
+  if (!aligned16(w->codes_d) || !aligned16(w->codebook_d)) return TQ_ERR_ALIGN;
+  return TQ_OK;
+}
+
+// Launch with the programmatic-stream-serialization attribute so that a
+// kernel may start its weight prefetch while the previous one finishes.
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+#ifdef TQ_NO_PDL
+  cfg.numAttrs = 0;  // build option: plain stream ordering
+#else
+  cfg.numAttrs = 1;
+#endif
+  TQ_CUDA(cudaLaunchKernelEx(&cfg, kernel, args...));
+  return TQ_OK;
+}
+
+// ---- decode-MMA configuration ------------------------------------------------
+
+using tq::DmmaParams;
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Columns of one partial-sum tile: 1 at batch 1 (hi+lo summed), else 8 * NT.
+int dmma_nt_for(int32_t m) {
+  if (m <= 8) return 1;
+  if (m <= 16) return 2;
+  if (m <= 32) return 4;
+  return 8;
+}
+constexpr int kDmmaMaxM = 64;  // one dmma launch covers up to 64 tokens
+
+struct DmmaWs {
+  size_t counters_off, partials_off, bytes;
+};
+
+// Every workspace starts with a fixed region of per-tile arrival counters
+// (kCounterBytes, so every call, whatever its shape, finds its counters in
+// the same zeroed bytes; each call leaves them zero).  Everything after it
+// (partial sums, activation scratch) is written before it is read.
+constexpr size_t kCounterBytes = 64 * 1024;
+constexpr int64_t kMaxTiles = kCounterBytes / 4;  // n <= 262144 rows per call
+
+DmmaWs dmma_ws_layout(int64_t n_total, int32_t k, int mc) {
+  const int64_t tiles = (n_total + 15) / 16;
+  const int64_t units = tiles * (k / 256);
+  const int64_t warps = units < tq::DMMA_MAX_WARPS ? units : tq::DMMA_MAX_WARPS;
+  DmmaWs w;
+  w.counters_off = 0;
+  w.partials_off = kCounterBytes;
+  w.bytes = w.partials_off + (size_t)warps * 2 * 16 * mc * sizeof(float);
+  return w;
+}
+
+// views: pick the largest replication that fits next to the activations.
+int dmma_lv_for(bool hilo, int32_t k) {
+  const size_t xs = hilo ? (size_t)k * 4 : 0;
+  const size_t limit = 227 * 1024;
+  for (int lv = 3; lv > 0; --lv)
+    if ((16384u << lv) + xs <= limit) return lv;
+  return 0;
+}
+
+template <int LV, int NT, bool HILO>
+int dmma_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream) {
+  auto kern = tq::dmma_kernel<LV, NT, HILO>;
+  const size_t smem = (16384u << LV) + (HILO ? (size_t)p.k * 4 : 0);
+  // per instantiation and device: opt in to large shared memory once and
+  // remember the occupancy for each shared-memory size class seen
+  static int occ_cache[kMaxDevices][64];
+  int dev = 0;
+  TQ_CUDA(cudaGetDevice(&dev));
+  const int cls = (int)(smem >> 12) & 63;
+  int occ = occ_cache[dev][cls];
+  if (occ == 0) {
+    TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
+    if (occ < 1) return TQ_ERR_SHAPE;
+    occ_cache[dev][cls] = occ;
+  }
+  int64_t grid = (int64_t)num_sms * occ;
+  const int64_t need = (p.units + tq::DMMA_WARPS - 1) / tq::DMMA_WARPS;
+  if (grid > need) grid = need;
+  if (grid * tq::DMMA_WARPS > tq::DMMA_MAX_WARPS) grid = tq::DMMA_MAX_WARPS / tq::DMMA_WARPS;
+  int64_t aw = grid * tq::DMMA_WARPS;
+  if (aw > p.units) aw = p.units;
+  p.active_warps = (int32_t)aw;
+  return launch(kern, dim3((unsigned)grid), dim3(tq::DMMA_THREADS), smem, stream, p);
+}
+
+template <int NT, bool HILO>
+int dmma_launch_lv(DmmaParams& p, int lv, int num_sms, cudaStream_t stream) {
+  switch (lv) {
+    case 3: return dmma_launch_t<3, NT, HILO>(p, num_sms, stream);
+    case 2: return dmma_launch_t<2, NT, HILO>(p, num_sms, stream);
+    case 1: return dmma_launch_t<1, NT, HILO>(p, num_sms, stream);
+    default: return dmma_launch_t<0, NT, HILO>(p, num_sms, stream);
+  }
+}
+
+// Fill the shape / workspace fields of p and launch.  p.m <= 64.
+int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
+  const int nt = hilo ? 1 : dmma_nt_for(p.m);
+  const int mc = hilo ? 1 : nt * 8;
+  const DmmaWs L = dmma_ws_layout(p.n_total, p.k, mc);
+  if (!ws) return TQ_ERR_WORKSPACE;
+  if (ws_bytes < L.bytes) return TQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return TQ_ERR_ALIGN;
+  p.tiles = (p.n_total + 15) / 16;
+  if (p.tiles > kMaxTiles) return TQ_ERR_SHAPE;
+  p.blocks = p.k / 256;
+  p.units = (int64_t)p.tiles * p.blocks;
+  p.counters = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.counters_off);
+  p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + L.partials_off);
+  const int lv = dmma_lv_for(hilo, p.k);
+  if (hilo) return dmma_launch_lv<1, true>(p, lv, num_sms, stream);
+  switch (nt) {
+    case 1: return dmma_launch_lv<1, false>(p, lv, num_sms, stream);
+    case 2: return dmma_launch_lv<2, false>(p, lv, num_sms, stream);
+    case 4: return dmma_launch_lv<4, false>(p, lv, num_sms, stream);
+    default: return dmma_launch_lv<8, false>(p, lv, num_sms, stream);
+  }
+}
+
+void dmma_single(DmmaParams& p, const tq_weight_t* w) {
+  memset(&p, 0, sizeof(p));
+  p.seg[0].codes = w->codes_d;
+  p.seg[0].scales = w->scales_d;
+  p.seg[0].rows = w->n;
+  p.seg[0].row0 = 0;
+  p.nseg = 1;
+  p.codebook = w->codebook_d;
+  p.n_total = w->n;
+  p.k = w->k;
+}
+
+// ---- layer stack helpers -------------------------------------------------------
+
+const double kScaleLo = 0.005, kScaleHi = 0.03;
+
+float stack_alpha(int32_t k) {
+  const double es2 = (kScaleHi * kScaleHi * kScaleHi - kScaleLo * kScaleLo * kScaleLo) / (3.0 * (kScaleHi - kScaleLo));
+  return (float)(1.0 / sqrt((double)k * es2));
+}
+
+// ops of phase p (first one is handed on)
+int phase_ops(const tq_layer_t* L, int phase, const tq_weight_t* ops[3]) {
+  switch (phase) {
+    case 0: ops[0] = &L->q; ops[1] = &L->k; ops[2] = &L->v; return 3;
+    case 1: ops[0] = &L->o; return 1;
+    case 2: ops[0] = &L->gate; ops[1] = &L->up; return 2;
+    case 3: ops[0] = &L->down; return 1;
+    default: return 0;
+  }
+}
+
+int phase_check(const tq_layer_t* L, int phase, int* nops, const tq_weight_t* ops[3], int64_t* n_total) {
+  if (!L) return TQ_ERR_NULL;
+  *nops = phase_ops(L, phase, ops);
+  if (*nops == 0) return TQ_ERR_SHAPE;
+  int64_t n = 0;
+  for (int i = 0; i < *nops; ++i) {
+    int st = check_weight(ops[i]);
+    if (st != TQ_OK) return st;
+    if (ops[i]->k != ops[0]->k || ops[i]->codebook_d != ops[0]->codebook_d) return TQ_ERR_SHAPE;
+    n += ops[i]->n;
+  }
+  if (n > 0x7fffffff) return TQ_ERR_SHAPE;
+  *n_total = n;
+  return TQ_OK;
+}
+
+// Workspace of one phase call at m tokens:
+//  [dmma counters + partials][x' fp16 [m][k] when m > 1]
+size_t phase_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
+  const int mc = (m <= 1) ? 1 : dmma_nt_for(m < kDmmaMaxM ? m : kDmmaMaxM) * 8;
+  size_t b = dmma_ws_layout(n_total, k, mc).bytes;
+  if (m > 1) b = round_up(b, 256) + round_up((size_t)m * k * 2, 256);
+  return b;
+}
+
+int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint64_t seed, float* y,
+              uint16_t* handoff, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
+  int nops = 0;
+  const tq_weight_t* ops[3];
+  int64_t n_total = 0;
+  int st = phase_check(L, phase, &nops, ops, &n_total);
+  if (st != TQ_OK) return st;
+  const int32_t k = ops[0]->k;
+  if (ws_bytes < phase_ws_bytes(n_total, k, m)) return TQ_ERR_WORKSPACE;
+  DmmaParams p;
+  memset(&p, 0, sizeof(p));
+  int32_t row0 = 0;
+  for (int i = 0; i < nops; ++i) {
+    p.seg[i].codes = ops[i]->codes_d;
+    p.seg[i].scales = ops[i]->scales_d;
+    p.seg[i].rows = ops[i]->n;
+    p.seg[i].row0 = row0;
+    row0 += ops[i]->n;
+  }
+  p.nseg = nops;
+  p.codebook = ops[0]->codebook_d;
+  p.n_total = (int32_t)n_total;
+  p.k = k;
+  p.y = y;
+  p.handoff = handoff;
+  p.handoff_rows = ops[0]->n;
+  p.alpha = stack_alpha(k);
+  if (m == 1) {
+    p.m = 1;
+    p.x_bf16 = x;
+    p.rht_seed = seed;
+    return dmma_run(p, true, ws, ws_bytes, num_sms, stream);
+  }
+  // m > 1: RHT to fp16 in the workspace tail, then the small-batch kernel in
+  // chunks of up to 64 tokens.
+  const size_t dm_bytes = round_up(dmma_ws_layout(n_total, k, dmma_nt_for(m < kDmmaMaxM ? m : kDmmaMaxM) * 8).bytes, 256);
+  uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + dm_bytes);
+  {
+    const int64_t tasks = (int64_t)m * (k / 512);
+    int64_t blocks = (tasks + 7) / 8;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    st = launch(tq::rht_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, x, (int)m, (int)k, seed,
+                (void*)xr);
+    if (st != TQ_OK) return st;
+  }
+  for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
+    DmmaParams pc = p;
+    pc.m = (m - t0) < kDmmaMaxM ? (m - t0) : kDmmaMaxM;
+    pc.x_f16 = xr + (size_t)t0 * k;
+    pc.y = y ? y + (size_t)t0 * n_total : nullptr;
+    pc.handoff = handoff ? handoff + (size_t)t0 * ops[0]->n : nullptr;
+    st = dmma_run(pc, false, ws, dm_bytes, num_sms, stream);
+    if (st != TQ_OK) return st;
+  }
+  return TQ_OK;
+}
+
+int64_t phase_n(const tq_layer_t* L, int phase) {
+  const tq_weight_t* ops[3];
+  int n = phase_ops(L, phase, ops);
+  int64_t t = 0;
+  for (int i = 0; i < n; ++i) t += ops[i]->n;
+  return t;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_pack_info(int32_t n, int32_t k, tq_pack_info_t* out) {
+  if (!out) return TQ_ERR_NULL;
+  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
+  out->n = n;
+  out->k = k;
+  out->group = 4;
+  out->block = 256;
+  out->rht_block = 512;
+  out->n_states = 8;
+  out->code_bytes = (int64_t)n * (k / 4);
+  out->scale_bytes = (int64_t)n * (k / 256) * 2;
+  out->codebook_bytes = 8 * 256 * 4 * 2;
+  out->packed_bytes = out->code_bytes + out->scale_bytes;
+  out->bits_per_weight = 8.0 * (double)out->packed_bytes / ((double)n * (double)k);
+  return TQ_OK;
+}
+
+int tq_decode(const tq_weight_t* w, uint16_t* w_f16_d, void* stream) {
+  int st = check_weight(w);
+  if (st != TQ_OK) return st;
+  if (!w_f16_d) return TQ_ERR_NULL;
+  if (!aligned16(w_f16_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  const int64_t groups = (int64_t)w->n * (w->k / 4);
+  int64_t blocks = (groups + 255) / 256;
+  if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+  return launch(tq::decode_kernel, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, w->codes_d, w->scales_d,
+                w->codebook_d, (int)w->n, (int)w->k, w_f16_d);
+}
+
+int tq_rht(const uint16_t* x_bf16_d, int32_t m, int32_t k, uint64_t seed, void* x_rot_d, int32_t out_dtype,
+           void* stream) {
+  if (m < 0 || !k_ok(k)) return TQ_ERR_SHAPE;
+  if (out_dtype != TQ_F32 && out_dtype != TQ_F16) return TQ_ERR_SHAPE;
+  if (m == 0) return TQ_OK;
+  if (!x_bf16_d || !x_rot_d) return TQ_ERR_NULL;
+  if (!aligned16(x_bf16_d) || !aligned16(x_rot_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  int st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  const int64_t tasks = (int64_t)m * (k / 512);
+  int64_t blocks = (tasks + 7) / 8;
+  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
+  if (out_dtype == TQ_F16)
+    return launch(tq::rht_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+                  (int)k, seed, x_rot_d);
+  return launch(tq::rht_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+                (int)k, seed, x_rot_d);
+}
+
+int tq_gemv_workspace(int32_t n, int32_t k, size_t* bytes) {
+  if (!bytes) return TQ_ERR_NULL;
+  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
+  *bytes = dmma_ws_layout(n, k, 1).bytes;
+  return TQ_OK;
+}
+
+int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* workspace_d, size_t ws_bytes,
+            void* stream) {
+  int st = check_weight(w);
+  if (st != TQ_OK) return st;
+  if (!x_rot_d || !y_d) return TQ_ERR_NULL;
+  if (!aligned16(x_rot_d) || !aligned16(y_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  DmmaParams p;
+  dmma_single(p, w);
+  p.m = 1;
+  p.x_f32 = x_rot_d;
+  p.y = y_d;
+  return dmma_run(p, true, workspace_d, ws_bytes, sms, (cudaStream_t)stream);
+}
+
+int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes) {
+  if (!bytes) return TQ_ERR_NULL;
+  if (n < 1 || !k_ok(k) || m < 0 || m > 4096) return TQ_ERR_SHAPE;
+  const int mm = m < 1 ? 1 : (m < kDmmaMaxM ? m : kDmmaMaxM);
+  *bytes = dmma_ws_layout(n, k, dmma_nt_for(mm) * 8).bytes;
+  return TQ_OK;
+}
+
+int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
+            size_t ws_bytes, void* stream) {
+  int st = check_weight(w);
+  if (st != TQ_OK) return st;
+  if (m < 0 || m > 4096) return TQ_ERR_SHAPE;
+  if (m == 0) return TQ_OK;
+  if (!x_rot_f16_d || !y_d) return TQ_ERR_NULL;
+  if (!aligned16(x_rot_f16_d) || !aligned16(y_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
+    DmmaParams p;
+    dmma_single(p, w);
+    p.m = (m - t0) < kDmmaMaxM ? (m - t0) : kDmmaMaxM;
+    p.x_f16 = x_rot_f16_d + (size_t)t0 * w->k;
+    p.y = y_d + (size_t)t0 * w->n;
+    st = dmma_run(p, false, workspace_d, ws_bytes, sms, (cudaStream_t)stream);
+    if (st != TQ_OK) return st;
+  }
+  return TQ_OK;
+}
+
+int tq_workspace_init(void* workspace_d, size_t bytes, void* stream) {
+  if (bytes == 0) return TQ_OK;
+  if (!workspace_d) return TQ_ERR_NULL;
+  TQ_CUDA(cudaMemsetAsync(workspace_d, 0, bytes, (cudaStream_t)stream));
+  return TQ_OK;
+}
+
+uint64_t tq_stack_phase_seed(uint64_t seed, int32_t layer, int32_t phase) {
+  const uint64_t tag = 0x516E0000ULL | ((uint64_t)(uint32_t)layer << 2) | (uint64_t)(uint32_t)phase;
+  return tq::mix64(seed ^ tq::mix64(tag));
+}
+
+int tq_layer_phase_workspace(const tq_layer_t* layer, int32_t phase, int32_t m, size_t* bytes) {
+  if (!bytes) return TQ_ERR_NULL;
+  if (m < 0 || m > 4096) return TQ_ERR_SHAPE;
+  int nops = 0;
+  const tq_weight_t* ops[3];
+  int64_t n_total = 0;
+  int st = phase_check(layer, phase, &nops, ops, &n_total);
+  if (st != TQ_OK) return st;
+  *bytes = phase_ws_bytes(n_total, ops[0]->k, m < 1 ? 1 : m);
+  return TQ_OK;
+}
+
+int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf16_d, int32_t m, uint64_t phase_seed,
+                   float* y_d, uint16_t* handoff_bf16_d, void* workspace_d, size_t ws_bytes, void* stream) {
+  if (m < 0 || m > 4096) return TQ_ERR_SHAPE;
+  int nops = 0;
+  const tq_weight_t* ops[3];
+  int64_t n_total = 0;
+  int st = phase_check(layer, phase, &nops, ops, &n_total);
+  if (st != TQ_OK) return st;
+  if (m == 0) return TQ_OK;
+  if (!x_bf16_d || !handoff_bf16_d || !workspace_d) return TQ_ERR_NULL;
+  if (!aligned16(x_bf16_d) || (y_d && !aligned16(y_d)) || !aligned16(workspace_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  return run_phase(layer, phase, x_bf16_d, m, phase_seed, y_d, handoff_bf16_d, workspace_d, ws_bytes, sms,
+                   (cudaStream_t)stream);
+}
+
+// Stack workspace: [phase workspace][y fp32 [m][max n]][a bf16 [m][q]]
+// [b bf16 [m][hidden]][c bf16 [m][inter]][h bf16 [m][hidden]]
+struct StackWs {
+  size_t phase, y, a, b, c, h, total;
+};
+
+static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, StackWs* L) {
+  if (!layers) return TQ_ERR_NULL;
+  if (n_layers < 1 || m < 1 || m > 4096) return TQ_ERR_SHAPE;
+  size_t phase = 0;
+  int64_t ymax = 0, amax = 0, bmax = 0, cmax = 0, hmax = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    for (int p = 0; p < 4; ++p) {
+      int nops = 0;
+      const tq_weight_t* ops[3];
+      int64_t n_total = 0;
+      int st = phase_check(&layers[l], p, &nops, ops, &n_total);
+      if (st != TQ_OK) return st;
+      size_t b = phase_ws_bytes(n_total, ops[0]->k, m);
+      if (b > phase) phase = b;
+      if (n_total > ymax) ymax = n_total;
+    }
+    const tq_layer_t& L0 = layers[l];
+    // the chain of shapes: h -> q|k|v (k = hidden) -> o (k = q.n) -> gate|up (k = o.n) -> down (k = gate.n)
+    if (L0.o.k != L0.q.n || L0.gate.k != L0.o.n || L0.down.k != L0.gate.n || L0.down.n != L0.q.k)
+      return TQ_ERR_SHAPE;
+    if (l > 0 && L0.q.k != layers[l - 1].down.n) return TQ_ERR_SHAPE;
+    if (L0.q.n > amax) amax = L0.q.n;
+    if (L0.o.n > bmax) bmax = L0.o.n;
+    if (L0.gate.n > cmax) cmax = L0.gate.n;
+    if (L0.down.n > hmax) hmax = L0.down.n;
+  }
+  L->phase = 0;
+  L->y = round_up(phase, 256);
+  L->a = L->y + round_up((size_t)m * ymax * 4, 256);
+  L->b = L->a + round_up((size_t)m * amax * 2, 256);
+  L->c = L->b + round_up((size_t)m * bmax * 2, 256);
+  L->h = L->c + round_up((size_t)m * cmax * 2, 256);
+  L->total = L->h + round_up((size_t)m * hmax * 2, 256);
+  return TQ_OK;
+}
+
+int tq_layer_stack_workspace(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t* bytes) {
+  if (!bytes) return TQ_ERR_NULL;
+  StackWs L;
+  int st = stack_layout(layers, n_layers, m, &L);
+  if (st != TQ_OK) return st;
+  *bytes = L.total;
+  return TQ_OK;
+}
+
+int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m, uint64_t seed,
+                   uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes, void* stream) {
+  if (m == 0) return TQ_OK;
+  StackWs L;
+  int st = stack_layout(layers, n_layers, m, &L);
+  if (st != TQ_OK) return st;
+  if (!h_in_bf16_d || !h_out_bf16_d || !workspace_d) return TQ_ERR_NULL;
+  if (!aligned16(h_in_bf16_d) || !aligned16(h_out_bf16_d) || !aligned16(workspace_d)) return TQ_ERR_ALIGN;
+  if (ws_bytes < L.total) return TQ_ERR_WORKSPACE;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  char* ws = static_cast<char*>(workspace_d);
+  float* y = reinterpret_cast<float*>(ws + L.y);
+  uint16_t* a = reinterpret_cast<uint16_t*>(ws + L.a);
+  uint16_t* b = reinterpret_cast<uint16_t*>(ws + L.b);
+  uint16_t* c = reinterpret_cast<uint16_t*>(ws + L.c);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  const size_t phase_bytes = L.y;
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int l = 0; l < n_layers; ++l) {
+    const uint16_t* in0 = (l == 0) ? h_in_bf16_d : h;
+    uint16_t* out3 = (l == n_layers - 1) ? h_out_bf16_d : h;
+    const uint16_t* ins[4] = {in0, a, b, c};
+    uint16_t* outs[4] = {a, b, c, out3};
+    for (int p = 0; p < 4; ++p) {
+      st = run_phase(&layers[l], p, ins[p], m, tq_stack_phase_seed(seed, l, p), y, outs[p], ws, phase_bytes, sms, s);
+      if (st != TQ_OK) return st;
+    }
+  }
+  return TQ_OK;
+}
+
+const char* tq_status_string(int status) {
+  switch (status) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_SHAPE: return "bad shape (k must be a positive multiple of 512, n >= 1, 0 <= m <= 4096)";
+    case TQ_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case TQ_ERR_NULL: return "required pointer is NULL";
+    case TQ_ERR_ARCH: return "device is not compute capability 10.0 (sm_100a)";
+    case TQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case TQ_ERR_CUDA: return "CUDA runtime error (see tq_last_cuda_error)";
+    case TQ_ERR_TIMEOUT: return "bounded device wait expired";
+    default: return "unknown status";
+  }
+}
+
+int tq_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

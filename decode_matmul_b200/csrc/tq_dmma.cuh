@@ -1,0 +1,427 @@
+// tq_dmma.cuh -- decode-in-registers matmul for batch 1 and small batches.
+//
+// Computes y[t][n] = sum_k W[n][k] x'[t][k] where W is decoded on the fly
+// from the trellis codes ("Pingala-8" landing page, "How it works"; "8 open
+// models" article, "Speed": at batch 1 the work is one read of the packed
+// weights per token).
+//
+// Design (B200, sm_100a):
+//  * Work unit = 16 weight rows x one 256-weight block (64 code bytes per
+//    row).  Units are ordered tile-major and split evenly over all active
+//    warps of the grid (contiguous ranges), so every SM gets the same number
+//    of code bytes whatever n and k are.  A tile whose units span several
+//    warps is summed by the last warp to arrive, in warp order (deterministic),
+//    through a small workspace of partial sums and per-tile counters.
+//  * Lane (g = lane/4, q = lane%4) streams 16 code bytes of row g and 16 of
+//    row g+8 (one 128-bit load each; 4 lanes cover a row's 64 codes), i.e. the
+//    m16n8k16 A-fragment owner of those rows.  The K order inside the MMA is
+//    permuted so that a lane's four A slots {2q,2q+1,2q+8,2q+9} hold the four
+//    weights of ONE code; B (the activations) uses the same permutation.
+//  * The state of code j is the low 3 bits of code j-1: the same 32-bit word
+//    or the previous word for 15 of 16 codes, the previous lane's last byte
+//    (one shuffle) for the first; lanes with q == 0 start a 256-block (state 0).
+//  * The codebook (16 KB) is replicated V times in shared memory as "views":
+//    entry e of view v lives at byte (e * 8V + 8v), so lanes with different
+//    v % V land in different bank pairs.  The gather is the in-core limit.
+//  * Decode is exact: W = fp16_RNE(scale * cb) by __hmul2, then mma.sync
+//    (fp16 x fp16 -> fp32).  Batch 1 takes fp32 x' and splits it into
+//    hi + lo fp16 columns of the MMA (x' = hi + lo to ~22 bits), so the fp32
+//    activation is not rounded to fp16.
+#pragma once
+
+#include "tq_common.cuh"
+#include "tq_rht.cuh"
+
+namespace tq {
+
+constexpr int DMMA_WARPS = 16;
+constexpr int DMMA_THREADS = DMMA_WARPS * 32;
+constexpr int DMMA_MAX_WARPS = 8192;  // bound on active warps (workspace sizing)
+
+struct DmmaSeg {
+  const uint8_t* codes;
+  const uint16_t* scales;
+  int32_t rows;
+  int32_t row0;  // first row of this segment in the concatenated output
+};
+
+struct DmmaParams {
+  DmmaSeg seg[3];
+  int32_t nseg;
+  const uint16_t* codebook;
+  int32_t n_total;
+  int32_t k;
+  int32_t m;
+  const float* x_f32;      // batch 1: x' fp32 [k]
+  const uint16_t* x_bf16;  // batch 1, fused RHT: x bf16 [k]
+  uint64_t rht_seed;
+  const uint16_t* x_f16;   // small batch: x' fp16 [m][k]
+  float* y;                // [m][n_total] or null
+  uint16_t* handoff;       // [m][handoff_rows] bf16 or null
+  int32_t handoff_rows;
+  float alpha;
+  float* partials;         // [active_warps][2][16 * MC]
+  int32_t* counters;       // [tiles]
+  int32_t tiles;
+  int32_t blocks;          // k / 256
+  int64_t units;           // tiles * blocks
+  int32_t active_warps;
+};
+
+__host__ __device__ __forceinline__ int64_t dmma_warp_begin(int64_t w, int64_t units, int64_t active) {
+  return (w * units) / active;
+}
+// The warp whose range contains unit u.
+__host__ __device__ __forceinline__ int64_t dmma_warp_of(int64_t u, int64_t units, int64_t active) {
+  return ((u + 1) * active + units - 1) / units - 1;
+}
+
+// Shared-memory offset of the hi (n=0) or lo (n=1) fp16 quad of group G,
+// arranged so that the 8 lanes reading one MMA step hit 64 contiguous bytes.
+__device__ __forceinline__ uint32_t xs_offset(int G, int n) {
+  return (uint32_t)((((((G >> 6) << 4) + (G & 15)) << 2) + ((G >> 4) & 3)) * 16 + n * 8);
+}
+
+__device__ __forceinline__ void store_hilo(uint8_t* xs, int G, float a, float b, float c, float d) {
+  uint32_t h0 = f2_to_h2(a, b), h1 = f2_to_h2(c, d);
+  float2 f0 = h2_to_f2(h0), f1 = h2_to_f2(h1);
+  uint32_t l0 = f2_to_h2(a - f0.x, b - f0.y), l1 = f2_to_h2(c - f1.x, d - f1.y);
+  *reinterpret_cast<uint2*>(xs + xs_offset(G, 0)) = make_uint2(h0, h1);
+  *reinterpret_cast<uint2*>(xs + xs_offset(G, 1)) = make_uint2(l0, l1);
+}
+
+struct DmmaChunk {
+  uint4 ca, cb;    // 16 code bytes of rows g and g+8
+  uint32_t sa, sb; // fp16 scales of rows g and g+8 (block b)
+};
+
+__device__ __forceinline__ void seg_lookup(const DmmaParams& p, int row, const uint8_t*& codes,
+                                           const uint16_t*& scales, int& local) {
+  int s = 0;
+  if (p.nseg > 1 && row >= p.seg[1].row0) s = 1;
+  if (p.nseg > 2 && row >= p.seg[2].row0) s = 2;
+  codes = s == 0 ? p.seg[0].codes : (s == 1 ? p.seg[1].codes : p.seg[2].codes);
+  scales = s == 0 ? p.seg[0].scales : (s == 1 ? p.seg[1].scales : p.seg[2].scales);
+  local = row - (s == 0 ? p.seg[0].row0 : (s == 1 ? p.seg[1].row0 : p.seg[2].row0));
+}
+
+// Pointers of this lane's two rows (g, g+8) of tile t at block 0: code bytes
+// of chunk q and the row's scales.  Rows past the end are clamped (their
+// results are never stored).
+struct DmmaRows {
+  const uint8_t* ca;
+  const uint8_t* cb;
+  const uint16_t* sa;
+  const uint16_t* sb;
+};
+
+__device__ __forceinline__ DmmaRows dmma_rows(const DmmaParams& p, int t, int g, int q) {
+  const int r0 = min(t * 16 + g, p.n_total - 1), r1 = min(t * 16 + g + 8, p.n_total - 1);
+  const uint8_t *c0, *c1;
+  const uint16_t *s0, *s1;
+  int l0, l1;
+  seg_lookup(p, r0, c0, s0, l0);
+  seg_lookup(p, r1, c1, s1, l1);
+  const int gpr = p.k >> 2;
+  DmmaRows r;
+  r.ca = c0 + (size_t)l0 * gpr + q * 16;
+  r.cb = c1 + (size_t)l1 * gpr + q * 16;
+  r.sa = s0 + (size_t)l0 * p.blocks;
+  r.sb = s1 + (size_t)l1 * p.blocks;
+  return r;
+}
+
+__device__ __forceinline__ DmmaChunk dmma_fetch(const DmmaRows& r, int b) {
+  DmmaChunk ch;
+  ch.ca = ldg_stream_u4(r.ca + b * 64);
+  ch.cb = ldg_stream_u4(r.cb + b * 64);
+  ch.sa = ldg_u16(r.sa + b);
+  ch.sb = ldg_u16(r.sb + b);
+  return ch;
+}
+
+// Offsets (bytes, relative to the views base) of the 4 codebook entries of
+// one 32-bit code word.  `r` is the byte-reversed word, `prev_hi` holds the
+// previous code in bits 0-7.  Entry e = (prev & 7) << 8 | code sits at
+// e << SH (+ view offset); the shifts put code at bit SH and prev at SH + 8.
+template <int SH>
+__device__ __forceinline__ void word_offsets(uint32_t r, uint32_t prev_hi, uint32_t vofs, uint32_t off[4]) {
+  constexpr uint32_t MASK = 0x7FFu << SH;
+  off[0] = (__funnelshift_r(r, prev_hi, 24 - SH) & MASK) | vofs;
+  off[1] = ((r >> (16 - SH)) & MASK) | vofs;
+  off[2] = ((r >> (8 - SH)) & MASK) | vofs;
+  off[3] = ((r << SH) & MASK) | vofs;
+}
+
+template <int NT, bool HILO>
+__device__ __forceinline__ void dmma_epilogue(const DmmaParams& p, int t, int g, int q, const float (&v)[NT][4]) {
+  const int R0 = t * 16 + g, R1 = R0 + 8;
+  if (HILO) {
+    if (q != 0) return;
+    const float y0 = v[0][0] + v[0][1], y1 = v[0][2] + v[0][3];
+    if (R0 < p.n_total) {
+      if (p.y) p.y[R0] = y0;
+      if (R0 < p.handoff_rows) p.handoff[R0] = f_to_bf16_bits(p.alpha * y0);
+    }
+    if (R1 < p.n_total) {
+      if (p.y) p.y[R1] = y1;
+      if (R1 < p.handoff_rows) p.handoff[R1] = f_to_bf16_bits(p.alpha * y1);
+    }
+  } else {
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tok = jt * 8 + 2 * q + e;
+        if (tok >= p.m) continue;
+        if (R0 < p.n_total) {
+          const float y = v[jt][e];
+          if (p.y) p.y[(size_t)tok * p.n_total + R0] = y;
+          if (R0 < p.handoff_rows) p.handoff[(size_t)tok * p.handoff_rows + R0] = f_to_bf16_bits(p.alpha * y);
+        }
+        if (R1 < p.n_total) {
+          const float y = v[jt][2 + e];
+          if (p.y) p.y[(size_t)tok * p.n_total + R1] = y;
+          if (R1 < p.handoff_rows) p.handoff[(size_t)tok * p.handoff_rows + R1] = f_to_bf16_bits(p.alpha * y);
+        }
+      }
+    }
+  }
+}
+
+// Element index (within a tile's 16 x MC partial) of accumulator value (jt, i).
+template <int NT, bool HILO>
+__device__ __forceinline__ int partial_index(int g, int q, int jt, int i) {
+  constexpr int MC = HILO ? 1 : NT * 8;
+  if (HILO) return (i < 2) ? g : g + 8;
+  const int row = (i < 2) ? g : g + 8;
+  return row * MC + jt * 8 + 2 * q + (i & 1);
+}
+
+template <int NT, bool HILO>
+__device__ __forceinline__ void dmma_flush(const DmmaParams& p, int64_t W, int64_t wb, int64_t we, int t, int g,
+                                           int q, float (&acc)[NT][4]) {
+  constexpr int MC = HILO ? 1 : NT * 8;
+  const int64_t B = p.blocks;
+  const int64_t t0 = (int64_t)t * B, t1 = t0 + B;
+  if (t0 >= wb && t1 <= we) {  // the whole tile ran in this warp
+    dmma_epilogue<NT, HILO>(p, t, g, q, acc);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int slot = (t == (int)(wb / B)) ? 0 : 1;
+  float* part = p.partials + ((size_t)W * 2 + slot) * (16 * MC);
+  if (HILO) {
+    if (q == 0) {
+      part[g] = acc[0][0] + acc[0][1];
+      part[g + 8] = acc[0][2] + acc[0][3];
+    }
+  } else {
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) part[partial_index<NT, HILO>(g, q, jt, i)] = acc[jt][i];
+  }
+  __threadfence();
+  __syncwarp();
+  int old = 0;
+  if (lane == 0) old = atomicAdd(p.counters + t, 1);
+  old = __shfl_sync(0xffffffffu, old, 0);
+  const int64_t wa = dmma_warp_of(t0, p.units, p.active_warps);
+  const int64_t wz = dmma_warp_of(t1 - 1, p.units, p.active_warps);
+  if (old != (int)(wz - wa)) return;  // not the last contributor
+  __threadfence();
+  // Sum the contributors in warp order.  Only the first contributor can have
+  // started before the tile (then the tile is its tail slot); every later one
+  // starts inside it (head slot).  Loads are issued CB contributors at a time.
+  constexpr int CB = NT >= 8 ? 1 : 8 / NT;
+  float sum[NT][4];
+#pragma unroll
+  for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sum[jt][i] = 0.f;
+  const int first_slot = (dmma_warp_begin(wa, p.units, p.active_warps) >= t0) ? 0 : 1;
+  const int ncontrib = (int)(wz - wa) + 1;
+  for (int c0 = 0; c0 < ncontrib; c0 += CB) {
+    float v[CB][NT][4];
+#pragma unroll
+    for (int c = 0; c < CB; ++c) {
+      const int cc = min(c0 + c, ncontrib - 1);
+      const int64_t w = wa + cc;
+      const int s = (cc == 0) ? first_slot : 0;
+      const float* src = p.partials + ((size_t)w * 2 + s) * (16 * MC);
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (HILO) {
+            v[c][jt][i] = (jt == 0 && (i == 0 || i == 2)) ? __ldcg(src + (i == 0 ? g : g + 8)) : 0.f;
+          } else {
+            v[c][jt][i] = __ldcg(src + partial_index<NT, HILO>(g, q, jt, i));
+          }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < CB; ++c)
+      if (c0 + c < ncontrib)
+#pragma unroll
+        for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sum[jt][i] += v[c][jt][i];
+  }
+  dmma_epilogue<NT, HILO>(p, t, g, q, sum);
+  if (lane == 0) p.counters[t] = 0;  // leave the counter ready for the next call
+}
+
+// LV = log2(number of codebook views); NT = number of 8-token MMA column
+// tiles (small batch); HILO = batch-1 mode with fp32 x' split in hi/lo.
+template <int LV, int NT, bool HILO>
+__global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_constant__ DmmaParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  constexpr int V = 1 << LV;
+  constexpr int SH = 3 + LV;
+  uint8_t* xs = smem + (16384 << LV);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, q = lane & 3;
+
+  pdl_launch_dependents();
+
+  // Codebook views (no kernel in the stream writes the codebook).
+  for (int e = tid; e < 2048; e += DMMA_THREADS) {
+    const uint2 ent = reinterpret_cast<const uint2*>(p.codebook)[e];
+    uint8_t* dst = smem + (e << SH);
+    if (V == 1) {
+      *reinterpret_cast<uint2*>(dst) = ent;
+    } else {
+#pragma unroll
+      for (int v = 0; v < V; v += 2)
+        *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(ent.x, ent.y, ent.x, ent.y);
+    }
+  }
+
+  const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
+  const bool active = W < p.active_warps;
+  const int64_t wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
+  const int64_t we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
+
+  // The weights are not written by any kernel of the stream: prefetch the
+  // first chunk before waiting on the previous kernel.
+  int t = 0, b = 0;  // tile and block of the current unit (no divisions in the loop)
+  DmmaRows rows;
+  DmmaChunk cur;
+  if (wb < we) {
+    t = (int)(wb / p.blocks);
+    b = (int)(wb - (int64_t)t * p.blocks);
+    rows = dmma_rows(p, t, g, q);
+    cur = dmma_fetch(rows, b);
+  }
+
+  pdl_wait();
+
+  if (HILO) {
+    if (p.x_bf16) {
+      for (int blk = warp; blk < p.k / 512; blk += DMMA_WARPS) {
+        float v[16];
+        rht512_warp(p.x_bf16, blk, p.rht_seed, v);
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4)
+          store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
+      }
+    } else {
+      for (int G = tid; G < (p.k >> 2); G += DMMA_THREADS) {
+        const float4 x = reinterpret_cast<const float4*>(p.x_f32)[G];
+        store_hilo(xs, G, x.x, x.y, x.z, x.w);
+      }
+    }
+  }
+  __syncthreads();
+  if (wb >= we) return;
+
+  const uint32_t vofs = (uint32_t)((lane & (V - 1)) << 3);
+  // two accumulator sets (even / odd code steps) halve the MMA dependency chain
+  float acc[NT][4], acc2[NT][4];
+#pragma unroll
+  for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
+
+  const int nunits = (int)(we - wb);
+  for (int iu = 0; iu < nunits; ++iu) {
+    int tn = t, bn = b + 1;
+    if (bn == p.blocks) {
+      bn = 0;
+      ++tn;
+    }
+    DmmaRows nrows = rows;
+    DmmaChunk nxt;
+    if (iu + 1 < nunits) {
+      if (bn == 0) nrows = dmma_rows(p, tn, g, q);
+      nxt = dmma_fetch(nrows, bn);
+    }
+
+    const uint8_t* xs_lane = xs + (((b << 4) << 2) + q) * 16 + (g & 1) * 8;
+    const uint16_t* xg_lane[NT];
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + 4 * (size_t)(b * 64 + q * 16);
+    // previous code byte of each row chunk (state of code 0); 0 at a block start
+    uint32_t pa = __shfl_up_sync(0xffffffffu, cur.ca.w, 1) >> 24;
+    uint32_t pb = __shfl_up_sync(0xffffffffu, cur.cb.w, 1) >> 24;
+    if (q == 0) pa = pb = 0;
+    const uint32_t wa[4] = {cur.ca.x, cur.ca.y, cur.ca.z, cur.ca.w};
+    const uint32_t wbw[4] = {cur.cb.x, cur.cb.y, cur.cb.z, cur.cb.w};
+    const uint32_t sa2 = cur.sa | (cur.sa << 16), sb2 = cur.sb | (cur.sb << 16);
+
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t ra = __byte_perm(wa[i], 0, 0x0123), rb = __byte_perm(wbw[i], 0, 0x0123);
+      const uint32_t ha = (i == 0) ? pa : __byte_perm(wa[i - 1], 0, 0x0123);
+      const uint32_t hb = (i == 0) ? pb : __byte_perm(wbw[i - 1], 0, 0x0123);
+      uint32_t oa[4], ob[4];
+      word_offsets<SH>(ra, ha, vofs, oa);
+      word_offsets<SH>(rb, hb, vofs, ob);
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = i * 4 + jj;
+        const uint2 ea = *reinterpret_cast<const uint2*>(smem + oa[jj]);
+        const uint2 eb = *reinterpret_cast<const uint2*>(smem + ob[jj]);
+        uint32_t a[4];
+        a[0] = hmul2_u32(ea.x, sa2);
+        a[2] = hmul2_u32(ea.y, sa2);
+        a[1] = hmul2_u32(eb.x, sb2);
+        a[3] = hmul2_u32(eb.y, sb2);
+        // B columns other than the live ones (hi/lo at batch 1, tokens < m
+        // otherwise) only feed C columns that are never read, so every lane
+        // loads a valid activation quad without predicates.
+        if (HILO) {
+          const uint2 bw = *reinterpret_cast<const uint2*>(xs_lane + j * 64);
+          mma_16816((j & 1) ? acc2[0] : acc[0], a, bw.x, bw.y);
+        } else {
+#pragma unroll
+          for (int jt = 0; jt < NT; ++jt) {
+            const uint2 bv = __ldg(reinterpret_cast<const uint2*>(xg_lane[jt] + 4 * j));
+            mma_16816((j & 1) ? acc2[jt] : acc[jt], a, bv.x, bv.y);
+          }
+        }
+      }
+    }
+
+    if (iu + 1 == nunits || bn == 0) {
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[jt][i] += acc2[jt][i];
+      dmma_flush<NT, HILO>(p, W, wb, we, t, g, q, acc);
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
+    }
+    t = tn;
+    b = bn;
+    rows = nrows;
+    cur = nxt;
+  }
+}
+
+}  // namespace tq

@@ -1,0 +1,98 @@
+// tq_rht.cuh -- randomized Walsh-Hadamard transform of activations.
+//
+// "Pingala-8" landing page, "How it works": a random Hadamard rotation is
+// applied before the weights are encoded; "Bonsai 2 27B" article, change of
+// basis: the rotation lives in the stored weights and the matching transform
+// runs on the activations at run time.  Here: x' = H_512 D x per 512-block,
+// H in natural (Sylvester) order, orthonormal (1/sqrt(512)), D = diag(+-1)
+// drawn from SplitMix64.
+//
+// One warp owns one 512-block of one row.  Lane l holds elements 16l..16l+15
+// in registers: index bits 0-3 are register bits, bits 4-8 are lane bits.
+// The 9 butterfly stages are 4 in-register stages and 5 shfl.xor stages.
+#pragma once
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+// In-place unnormalised Sylvester transform of the 512 values held by a warp.
+__device__ __forceinline__ void wht512_warp(float v[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (!(r & h)) {
+        float a = v[r], b = v[r | h];
+        v[r] = a + b;
+        v[r | h] = a - b;
+      }
+    }
+  }
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      float o = __shfl_xor_sync(0xffffffffu, v[r], m);
+      v[r] = upper ? (o - v[r]) : (v[r] + o);
+    }
+  }
+}
+
+// Load this lane's 16 bf16 inputs of block `blk` of row `x_row`, apply D,
+// transform, scale by 1/sqrt(512).  Returns values for elements 16*lane + r.
+__device__ __forceinline__ void rht512_warp(const uint16_t* __restrict__ x_row, int blk, uint64_t seed,
+                                            float v[16]) {
+  const int lane = threadIdx.x & 31;
+  const int base = blk * 512 + lane * 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x_row + base);
+  uint4 p0 = src[0], p1 = src[1];
+  uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t lo = w[i] & 0xFFFFu, hi = w[i] >> 16;
+    uint32_t k0 = (uint32_t)(base + 2 * i), k1 = k0 + 1;
+    // D: flip the sign bit of the bf16 value where d[k] = -1 (exact)
+    if (rht_sign_negative(seed, k0)) lo ^= 0x8000u;
+    if (rht_sign_negative(seed, k1)) hi ^= 0x8000u;
+    v[2 * i] = bf16_bits_to_f(lo);
+    v[2 * i + 1] = bf16_bits_to_f(hi);
+  }
+  wht512_warp(v);
+  const float inv = 0.044194173824159216f;  // 1/sqrt(512)
+#pragma unroll
+  for (int r = 0; r < 16; ++r) v[r] *= inv;
+}
+
+// Standalone RHT: grid-stride over (row, block) warp tasks.
+template <bool OUT_F16>
+__global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x, int m, int k, uint64_t seed,
+                                                  void* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  const int blocks = k / 512;
+  const long long tasks = (long long)m * blocks;
+  const int lane = threadIdx.x & 31;
+  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long t = warp0; t < tasks; t += nwarps) {
+    const int row = (int)(t / blocks), blk = (int)(t % blocks);
+    float v[16];
+    rht512_warp(x + (size_t)row * k, blk, seed, v);
+    const size_t o = (size_t)row * k + (size_t)blk * 512 + lane * 16;
+    if (OUT_F16) {
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + o);
+      dst[0] = make_uint4(f2_to_h2(v[0], v[1]), f2_to_h2(v[2], v[3]), f2_to_h2(v[4], v[5]), f2_to_h2(v[6], v[7]));
+      dst[1] = make_uint4(f2_to_h2(v[8], v[9]), f2_to_h2(v[10], v[11]), f2_to_h2(v[12], v[13]),
+                          f2_to_h2(v[14], v[15]));
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+  }
+}
+
+}  // namespace tq

@@ -1,0 +1,207 @@
+/*
+ * tq.h -- C ABI of libtq, the B200 (sm_100a) trellis-decode matmul library.
+ *
+ * The method (pages cited by title and section):
+ *   "Pingala-8" landing page, "How it works": linear-layer weights are stored
+ *   as an 8-state trellis code over groups of 4 weights, coded in order; a
+ *   small state carried from one group to the next selects the set of values
+ *   the next group may use.  A random Hadamard rotation is applied to the
+ *   weights before encoding.
+ *   "Bonsai 2 27B" article, change-of-basis paragraph: the rotation is folded
+ *   into the stored weights; the matching transform runs on the activations
+ *   at inference time.
+ *   "8 open models ... what 2-bit quantization costs", "Size": per-block
+ *   scales add bits on top of the 2-bit codes; "Speed": batch-1 decoding is
+ *   a matter of reading the weights from memory once per token.
+ *
+ * Format (the pages fix no bit layout; this is the layout the library uses):
+ *   codes     uint8  [n][k/4]   one code c per group of 4 weights, row-major
+ *   scales    fp16   [n][k/256] one scale per row and 256-weight block
+ *   codebook  fp16   [8][256][4] entry (s, c) is a 4-vector
+ *   state     s_g = 0 when g % 64 == 0, else codes[n][g-1] & 7
+ *   weight    W[n][4g+j] = fp16_RNE(scale[n][g/64] * codebook[s_g][c_g][j])
+ *   size      n*k/4 + 2*n*k/256 bytes = 2.0625 bits per weight
+ *   RHT       x'[m][512b+i] = (1/sqrt(512)) sum_j H[i][j] d[512b+j] x[m][512b+j],
+ *             H[i][j] = (-1)^popcount(i&j) (natural / Sylvester order),
+ *             d[k] = -1 if bit 63 of splitmix64_k(seed) is set, else +1,
+ *             where splitmix64_k(seed) is the k-th (0-based) output of a
+ *             SplitMix64 generator whose state starts at `seed`.
+ *   linear    y[m][n] = sum_k W[n][k] x'[m][k]   (fp32 output)
+ *
+ * Conventions for every call:
+ *   - Pointers named *_d are DEVICE pointers and are caller-owned; the library
+ *     never allocates device memory and never frees what it is given.
+ *     Host pointers (structs, `out` arguments) are read or written before the
+ *     call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous on it; none synchronises.
+ *   - Return value: TQ_OK or one TQ_ERR_* code.  On an error nothing is
+ *     launched.  No C++ exception crosses this interface.
+ *   - k must be a positive multiple of 512.  n >= 1.  m >= 0 (m == 0 and
+ *     n == 0 are accepted as empty work and return TQ_OK without a launch
+ *     where stated).
+ *   - codes_d, x and y pointers must be 16-byte aligned (TQ_ERR_ALIGN).
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define TQ_OK 0
+#define TQ_ERR_SHAPE 1     /* a size is out of range (k % 512, n < 1, m < 0, m too large) */
+#define TQ_ERR_ALIGN 2     /* a pointer is not 16-byte aligned */
+#define TQ_ERR_NULL 3      /* a required pointer is NULL */
+#define TQ_ERR_ARCH 4      /* the current device is not compute capability 10.0 */
+#define TQ_ERR_WORKSPACE 5 /* workspace missing or smaller than the *_workspace query */
+#define TQ_ERR_CUDA 6      /* a CUDA runtime call failed; tq_last_cuda_error() has its code */
+#define TQ_ERR_TIMEOUT 7   /* a bounded device-side wait expired (reported by the status word) */
+
+/* output element types */
+#define TQ_F32 0
+#define TQ_F16 1
+
+/* One trellis-coded weight.  All pointers are device pointers (caller-owned).
+ * codes_d: uint8 [n][k/4], 16-byte aligned.  scales_d: fp16 bits [n][k/256].
+ * codebook_d: fp16 bits [8][256][4] (16384 bytes), 16-byte aligned. */
+typedef struct tq_weight {
+  const uint8_t* codes_d;
+  const uint16_t* scales_d;
+  const uint16_t* codebook_d;
+  int32_t n;
+  int32_t k;
+} tq_weight_t;
+
+/* Sizes of one packed n x k weight ("Size" section: codes plus per-block
+ * scales).  packed_bytes = code_bytes + scale_bytes = n*k*33/128. */
+typedef struct tq_pack_info {
+  int32_t n, k;
+  int32_t group;     /* 4 weights per code */
+  int32_t block;     /* 256 weights per scale and per state reset */
+  int32_t rht_block; /* 512 */
+  int32_t n_states;  /* 8 */
+  int64_t code_bytes;
+  int64_t scale_bytes;
+  int64_t codebook_bytes; /* 16384, shared by all rows */
+  int64_t packed_bytes;
+  double bits_per_weight; /* 2.0625 */
+} tq_pack_info_t;
+
+/* Host-only.  Fills *out for an n x k weight.  TQ_ERR_SHAPE unless n >= 1 and
+ * k is a positive multiple of 512; TQ_ERR_NULL if out is NULL. */
+TQ_API int tq_pack_info(int32_t n, int32_t k, tq_pack_info_t* out);
+
+/* Decode the whole weight to fp16 (test and inspection export; the matmul
+ * calls never materialise W).  Definition: the "weight" line of the format
+ * above ("How it works": the previous group's state selects the codebook).
+ * w_f16_d: device, fp16 bits [n][k], caller-owned, 16-byte aligned. */
+TQ_API int tq_decode(const tq_weight_t* w, uint16_t* w_f16_d, void* stream);
+
+/* Randomized Hadamard transform of the activations ("How it works" and the
+ * "Bonsai 2" change-of-basis paragraph): x' = H_512 . D . x on each block of
+ * 512 features of each of the m rows.
+ * x_bf16_d: device bf16 bits [m][k], 16-byte aligned.
+ * x_rot_d:  device [m][k], fp32 (out_dtype TQ_F32) or fp16 (TQ_F16, rounded
+ *           to nearest even), 16-byte aligned.
+ * m == 0 returns TQ_OK without a launch. */
+TQ_API int tq_rht(const uint16_t* x_bf16_d, int32_t m, int32_t k, uint64_t seed, void* x_rot_d, int32_t out_dtype,
+           void* stream);
+
+/* Bytes of device workspace tq_gemv needs for an n x k weight (split-row
+ * partial sums and per-tile arrival counters). */
+TQ_API int tq_gemv_workspace(int32_t n, int32_t k, size_t* bytes);
+
+/* Batch-1 decode-GEMV: y[n] = sum_k W[n][k] x_rot[k] with W decoded on the
+ * fly from the codes ("Speed": one read of the packed weight per token).
+ * x_rot_d: device fp32 [k] (already rotated, e.g. by tq_rht), 16-byte aligned.
+ * y_d: device fp32 [n], 16-byte aligned.
+ * workspace_d: device, >= tq_gemv_workspace bytes, 16-byte aligned.  Every
+ * workspace begins with a 64 KB region of per-tile counters that must be zero
+ * before the first call (tq_workspace_init); every call of this library leaves
+ * it zero again, so one workspace may serve calls of any shape in turn.  The
+ * rest is scratch.  Calls that share a workspace must not overlap on the GPU.
+ * n is limited to 262144 rows per call (TQ_ERR_SHAPE). */
+TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* workspace_d, size_t ws_bytes,
+            void* stream);
+
+/* Bytes of device workspace tq_gemm needs for an n x k weight and m tokens. */
+TQ_API int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes);
+
+/* Small-batch / prompt matmul: y[t][n] = sum_k W[n][k] x_rot[t][k] for m
+ * tokens.  x_rot_f16_d: device fp16 [m][k] (tq_rht with TQ_F16), 16-byte
+ * aligned.  y_d: device fp32 [m][n], 16-byte aligned.  The kernel is chosen by
+ * m: register-decode warp MMAs for small m, decode-to-shared-memory tcgen05
+ * MMAs with TMEM accumulators for large m.  Same workspace rules as tq_gemv.
+ * m == 0 returns TQ_OK without a launch; m > 4096 is TQ_ERR_SHAPE. */
+TQ_API int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
+            size_t ws_bytes, void* stream);
+
+/* Zero a workspace (cudaMemsetAsync on `stream`). */
+TQ_API int tq_workspace_init(void* workspace_d, size_t bytes, void* stream);
+
+/* ---- layer stack ----------------------------------------------------------
+ * One layer = q, k, v, o, gate, up, down.  Per layer, four phases run in
+ * order; each starts with the RHT of its input and ends with the handoff
+ * h' = bf16_RNE(alpha(k_op) * y_op) of one op's output, where
+ * alpha(k) = 1/sqrt(k * E[s^2]) and E[s^2] = (0.03^3 - 0.005^3)/(3*0.025)
+ * (the second moment of a U[0.005, 0.03] scale), so that every handoff has
+ * about unit variance:
+ *   phase 0: x' = RHT(h)        -> q, k, v       handoff alpha(k_q) * q
+ *   phase 1: x' = RHT(phase 0)  -> o             handoff alpha(k_o) * o
+ *   phase 2: x' = RHT(phase 1)  -> gate, up      handoff alpha(k_gate) * gate
+ *   phase 3: x' = RHT(phase 2)  -> down          handoff alpha(k_down) * down = next h
+ * The k, v and up outputs are computed (and written to y) but not consumed:
+ * they stand in for attention and the gated product, which are not part of
+ * the trellis-decode path.  The RHT of phase p of layer l uses the seed
+ * tq_stack_phase_seed(seed, l, p).  All ops of one phase must share k and the
+ * codebook pointer (TQ_ERR_SHAPE otherwise). */
+typedef struct tq_layer {
+  tq_weight_t q, k, v, o, gate, up, down;
+} tq_layer_t;
+
+/* mix64(seed ^ mix64(0x516E0000 | layer << 2 | phase)), mix64 = the
+ * SplitMix64 output function. */
+TQ_API uint64_t tq_stack_phase_seed(uint64_t seed, int32_t layer, int32_t phase);
+
+/* Workspace bytes for one phase / for a whole stack at m tokens. */
+TQ_API int tq_layer_phase_workspace(const tq_layer_t* layer, int32_t phase, int32_t m, size_t* bytes);
+TQ_API int tq_layer_stack_workspace(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t* bytes);
+
+/* One phase of one layer.
+ * x_bf16_d: device bf16 [m][k_phase] input.
+ * y_d: device fp32 [m][n_phase] (the phase's ops concatenated in the order
+ *      listed above), or NULL to skip writing it.
+ * handoff_bf16_d: device bf16 [m][n_handoff] (n of q / o / gate / down).
+ * phase_seed: the RHT seed of this phase. */
+TQ_API int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf16_d, int32_t m, uint64_t phase_seed,
+                   float* y_d, uint16_t* handoff_bf16_d, void* workspace_d, size_t ws_bytes, void* stream);
+
+/* The whole stack: h_out = layers[n-1] o ... o layers[0] (h_in).
+ * layers: HOST array of n_layers tq_layer_t (device pointers inside).
+ * h_in_bf16_d / h_out_bf16_d: device bf16 [m][hidden]; they may alias.
+ * Enqueues 4 phases per layer on `stream` (capturable in a CUDA graph). */
+TQ_API int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m, uint64_t seed,
+                   uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes, void* stream);
+
+/* Human-readable text of a status code (static storage). */
+TQ_API const char* tq_status_string(int status);
+
+/* The cudaError_t value behind the last TQ_ERR_CUDA returned on this thread. */
+TQ_API int tq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

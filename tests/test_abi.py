@@ -1,0 +1,92 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and its host-only logic (sizes, argument checks, seeds) is right."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_matmul_b200 as tq
+import oracle
+import tqsynth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^TQ_API\s+[\w\s\*]+?\b(tq_\w+)\(", txt, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 15
+    L = tq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(tq.EXPORTS) <= set(names)
+
+
+@pytest.mark.parametrize("n,k", [(1024, 1024), (4096, 2560), (1024, 2560), (2560, 4096), (9728, 2560),
+                                 (2560, 9728), (14336, 4096), (4096, 14336), (6144, 5120), (5120, 6144),
+                                 (17408, 5120), (5120, 17408)])
+def test_pack_info_size_invariant(n, k):
+    info = tq.tq_pack_info(n, k)
+    assert info["packed_bytes"] * 128 == n * k * 33
+    assert info["packed_bytes"] == tqsynth.pack_bytes(n, k)
+    assert info["bits_per_weight"] == 2.0625
+    assert (info["group"], info["block"], info["rht_block"], info["n_states"]) == (4, 256, 512, 8)
+    assert info["codebook_bytes"] == 16384
+    c = tqsynth.codes(0, 0, 0, 2, k)
+    assert c.nbytes // 2 * n == info["code_bytes"]
+
+
+def test_pack_info_rejects_bad_shapes():
+    for n, k in [(0, 512), (-1, 512), (16, 0), (16, 256), (16, 1000), (16, -512)]:
+        with pytest.raises(tq.TqError) as e:
+            tq.tq_pack_info(n, k)
+        assert e.value.status == tq.TQ_ERR_SHAPE
+    assert tq.lib().tq_pack_info(16, 512, None) == tq.TQ_ERR_NULL
+
+
+def test_stack_workspace_sizes_monotone():
+    assert tq.tq_gemv_workspace(1024, 1024) > 0
+    assert tq.tq_gemm_workspace(1024, 1024, 64) >= tq.tq_gemm_workspace(1024, 1024, 1)
+    with pytest.raises(tq.TqError):
+        tq.tq_gemm_workspace(1024, 1024, 5000)
+
+
+def test_argument_checks_before_any_device_call():
+    L = tq.lib()
+    W = tq.tq_weight_t(16, 16, 16, 32, 512)  # fake, aligned addresses; never dereferenced
+    # shape errors
+    bad = tq.tq_weight_t(16, 16, 16, 32, 500)
+    assert L.tq_gemv(ctypes.byref(bad), 16, 16, 16, 1 << 20, None) == tq.TQ_ERR_SHAPE
+    assert L.tq_gemm(ctypes.byref(W), 16, -1, 16, 16, 1 << 20, None) == tq.TQ_ERR_SHAPE
+    assert L.tq_rht(16, 1, 500, 0, 16, tq.TQ_F32, None) == tq.TQ_ERR_SHAPE
+    assert L.tq_rht(16, 1, 512, 0, 16, 7, None) == tq.TQ_ERR_SHAPE
+    # null / alignment
+    assert L.tq_gemv(None, 16, 16, 16, 1 << 20, None) == tq.TQ_ERR_NULL
+    assert L.tq_gemv(ctypes.byref(W), None, 16, 16, 1 << 20, None) == tq.TQ_ERR_NULL
+    assert L.tq_gemv(ctypes.byref(W), 18, 16, 16, 1 << 20, None) == tq.TQ_ERR_ALIGN
+    mis = tq.tq_weight_t(17, 16, 16, 32, 512)
+    assert L.tq_decode(ctypes.byref(mis), 16, None) == tq.TQ_ERR_ALIGN
+    assert L.tq_rht(18, 1, 512, 0, 16, tq.TQ_F32, None) == tq.TQ_ERR_ALIGN
+    # empty work is fine and launches nothing
+    assert L.tq_rht(16, 0, 512, 0, 16, tq.TQ_F32, None) == tq.TQ_OK
+    assert L.tq_gemm(ctypes.byref(W), 16, 0, 16, 16, 1 << 20, None) == tq.TQ_OK
+
+
+def test_stack_phase_seed_matches_oracle():
+    # both sides implement SplitMix64 from its published definition
+    for s, l, p in [(0, 0, 0), (0, 35, 3), (12345, 7, 2), (2 ** 64 - 1, 63, 1)]:
+        assert tq.tq_stack_phase_seed(s, l, p) == oracle.stack_phase_seed(s, l, p)
+
+
+def test_status_strings():
+    for st in range(8):
+        assert len(tq.lib().tq_status_string(st)) > 0
