@@ -16,13 +16,14 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
-TQ_OK, TQ_ERR_SHAPE, TQ_ERR_ALIGN, TQ_ERR_NULL, TQ_ERR_ARCH, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_TIMEOUT = range(8)
+(TQ_OK, TQ_ERR_SHAPE, TQ_ERR_ALIGN, TQ_ERR_NULL, TQ_ERR_ARCH, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_TIMEOUT,
+ TQ_ERR_SCRATCH) = range(9)
 TQ_F32, TQ_F16 = 0, 1
 OPS = ("q", "k", "v", "o", "gate", "up", "down")
 
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
-           "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error")
+           "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc")
 
 
 class TqError(RuntimeError):
@@ -69,6 +70,7 @@ def _lib():
             "tq_rht": ([vp, i32, i32, u64, vp, i32, vp], ctypes.c_int),
             "tq_gemv_workspace": ([i32, i32, szp], ctypes.c_int),
             "tq_gemv": ([W, vp, vp, vp, sz, vp], ctypes.c_int),
+            "tq_gemv_noalloc": ([W, vp, vp, vp], ctypes.c_int),
             "tq_gemm_workspace": ([i32, i32, i32, szp], ctypes.c_int),
             "tq_gemm": ([W, vp, i32, vp, vp, sz, vp], ctypes.c_int),
             "tq_workspace_init": ([vp, sz, vp], ctypes.c_int),
@@ -189,6 +191,14 @@ def tq_gemv(w: DeviceWeight, x_rot, y=None, ws=None, stream=None):
         ws = workspace(tq_gemv_workspace(w.n, w.k), x_rot.device, stream)
     s = w.struct()
     _ok(_lib().tq_gemv(ctypes.byref(s), _ptr(x_rot), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "tq_gemv")
+    return y
+
+
+def tq_gemv_noalloc(w: DeviceWeight, x_rot, y, stream=None):
+    """Batch-1 GEMV with the library's built-in scratch (no workspace); y must
+    be given, so this call allocates nothing."""
+    s = w.struct()
+    _ok(_lib().tq_gemv_noalloc(ctypes.byref(s), _ptr(x_rot), _ptr(y), _stream(stream)), "tq_gemv_noalloc")
     return y
 
 

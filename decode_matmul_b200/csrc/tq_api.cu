@@ -547,6 +547,46 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
   return TQ_OK;
 }
 
+// ---- batch-1 GEMV with built-in scratch ---------------------------------------
+// For callers that cannot hand the library device memory.  The scratch lives
+// in a file-scope device array; host code only ever passes its device address,
+// which cudaGetSymbolAddress returns for the current device.
+
+static __device__ __align__(256) unsigned char g_gemv_scratch[TQ_GEMV_NOALLOC_SCRATCH_BYTES];
+static void* g_gemv_scratch_addr[kMaxDevices];  // device address of g_gemv_scratch, per device
+
+static_assert(TQ_GEMV_NOALLOC_SCRATCH_BYTES >= kCounterBytes + (size_t)tq::DMMA_MAX_WARPS * 2 * 16 * sizeof(float),
+              "built-in scratch must hold the counters and the batch-1 partial sums");
+
+int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* stream) {
+  int st = check_weight(w);
+  if (st != TQ_OK) return st;
+  if (!x_rot_d || !y_d) return TQ_ERR_NULL;
+  if (!aligned16(x_rot_d) || !aligned16(y_d)) return TQ_ERR_ALIGN;
+  if ((int64_t)(w->n + 15) / 16 > kMaxTiles || dmma_ws_layout(w->n, w->k, 1).bytes > TQ_GEMV_NOALLOC_SCRATCH_BYTES)
+    return TQ_ERR_SCRATCH;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  int dev = 0;
+  TQ_CUDA(cudaGetDevice(&dev));
+  if (!g_gemv_scratch_addr[dev]) {  // first call on this device: look up the array's device address
+    void* addr = nullptr;
+    TQ_CUDA(cudaGetSymbolAddress(&addr, g_gemv_scratch));
+    g_gemv_scratch_addr[dev] = addr;
+  }
+  void* ws = g_gemv_scratch_addr[dev];
+  cudaStream_t s = (cudaStream_t)stream;
+  // the arrival counters must start at zero whatever an earlier call left
+  TQ_CUDA(cudaMemsetAsync(ws, 0, kCounterBytes, s));
+  DmmaParams p;
+  dmma_single(p, w);
+  p.m = 1;
+  p.x_f32 = x_rot_d;
+  p.y = y_d;
+  return dmma_run(p, true, ws, TQ_GEMV_NOALLOC_SCRATCH_BYTES, sms, s);
+}
+
 const char* tq_status_string(int status) {
   switch (status) {
     case TQ_OK: return "ok";
@@ -557,6 +597,7 @@ const char* tq_status_string(int status) {
     case TQ_ERR_WORKSPACE: return "workspace missing or too small";
     case TQ_ERR_CUDA: return "CUDA runtime error (see tq_last_cuda_error)";
     case TQ_ERR_TIMEOUT: return "bounded device wait expired";
+    case TQ_ERR_SCRATCH: return "problem larger than the built-in scratch of tq_gemv_noalloc (n > 262144)";
     default: return "unknown status";
   }
 }

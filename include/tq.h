@@ -67,6 +67,7 @@ extern "C" {
 #define TQ_ERR_WORKSPACE 5 /* workspace missing or smaller than the *_workspace query */
 #define TQ_ERR_CUDA 6      /* a CUDA runtime call failed; tq_last_cuda_error() has its code */
 #define TQ_ERR_TIMEOUT 7   /* a bounded device-side wait expired (reported by the status word) */
+#define TQ_ERR_SCRATCH 8   /* the problem does not fit the built-in scratch of tq_gemv_noalloc */
 
 /* output element types */
 #define TQ_F32 0
@@ -134,6 +135,27 @@ TQ_API int tq_gemv_workspace(int32_t n, int32_t k, size_t* bytes);
  * n is limited to 262144 rows per call (TQ_ERR_SHAPE). */
 TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* workspace_d, size_t ws_bytes,
             void* stream);
+
+/* Batch-1 decode-GEMV that allocates nothing and takes no workspace.
+ * No counterpart on the pages: this is an interface for callers that cannot
+ * give the library device memory -- for example a runtime that owns every
+ * device allocation and has no workspace hook for a custom op, or a latency
+ * path that must not call cudaMalloc (which can synchronise the device).
+ * Same arguments and result as tq_gemv, without the workspace.
+ * Scratch: a file-scope device array of TQ_GEMV_NOALLOC_SCRATCH_BYTES
+ * (1 MiB + 64 KiB), which every GPU that loads the library holds until the
+ * process exits.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) for that device; make that first call before
+ * any stream capture.  Each call clears the array's counter region on
+ * `stream` before the kernel, and calls no cudaMalloc, cudaFree or other
+ * allocating routine.  Every call on a device shares that device's copy of
+ * the array, which keeps the last call's contents: calls that overlap on the
+ * GPU (for example on two streams) race and give wrong results, so run them
+ * one after another.
+ * Limit: n <= 262144 rows (TQ_ERR_SCRATCH beyond it); k any positive
+ * multiple of 512. */
+#define TQ_GEMV_NOALLOC_SCRATCH_BYTES ((size_t)(1u << 20) + (size_t)(64u << 10))
+TQ_API int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* stream);
 
 /* Bytes of device workspace tq_gemm needs for an n x k weight and m tokens. */
 TQ_API int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes);
