@@ -345,6 +345,8 @@ def main():
     bytes_step_layer = sum(pb)
     kern_ms_layer = sum(ph_ms)
     achieved = bytes_step_layer / (kern_ms_layer * 1e-3) / 1e9
+    flops_layer = 2.0 * m * shape.weights_per_layer()
+    tensor_tflops = flops_layer / (kern_ms_layer * 1e-3) / 1e12
     tokens = m * world * args.steps
     value = tokens / (ms_max * args.steps * 1e-3)
 
@@ -385,21 +387,27 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic: seeded random codes/scales/codebook/activations",
         "config": {"workload": f"{shape.name} stack, {shape.layers} layers, batch {m}", "layers": shape.layers,
                    "batch": m, "hidden": shape.hidden, "inter": shape.inter, "seed": 0,
                    "packed_bytes": shape.packed_bytes(), "parallelism": f"replicas x{world}",
                    "l2": "no flush: 937 MB-5.6 GB of resident weights per step exceed the 126 MB L2"},
         "compressed_weight_gbs": bytes_token * value / world / 1e9,
         "hbm_frac_of_measured": bytes_token * value / world / 1e9 / hbm,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_src,
-                     "kernel": "dmma_kernel (fused RHT + decode + mma.sync), all 4 phases",
-                     "phase_ms": ph_ms, "phase_bytes": pb},
+        "roofline": ({"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                      "frac": achieved / hbm, "traffic": None, "peak_source": peak_src,
+                      "kernel": "dmma_kernel (fused RHT + decode + mma.sync), all 4 phases",
+                      "phase_ms": ph_ms, "phase_bytes": pb} if m < 64 else
+                     {"bound": "tensor", "achieved": tensor_tflops, "peak": tflops, "unit": "TFLOP/s",
+                      "frac": tensor_tflops / tflops, "traffic": None, "peak_source": peak_src,
+                      "kernel": "rht_kernel + umma_kernel (tcgen05 decode-to-smem GEMM), all 4 phases",
+                      "phase_ms": ph_ms, "phase_flops": [2.0 * m * sum(n * k for o, n, k in shape.ops() if o in g)
+                                                         for g in (("q", "k", "v"), ("o",), ("gate", "up"),
+                                                                   ("down",))]}),
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": "tok/s", "h2d_bytes_per_step": int(h_host.numel() * 2),
                 "d2h_bytes_per_step": int(o_host.numel() * 2)},
-        "gpu_launches": 4 * shape.layers * args.steps * (1 if m == 1 else 1 + math.ceil(m / 64)),
+        "gpu_launches": 4 * shape.layers * args.steps * (1 if m == 1 else (2 if m >= 64 else 1 + math.ceil(m / 64))),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

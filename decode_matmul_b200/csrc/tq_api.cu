@@ -9,6 +9,9 @@
 #include "tq_decode.cuh"
 #include "tq_dmma.cuh"
 #include "tq_rht.cuh"
+#include "tq_umma.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace {
 
@@ -105,7 +108,7 @@ struct DmmaWs {
 // the same zeroed bytes; each call leaves them zero).  Everything after it
 // (partial sums, activation scratch) is written before it is read.
 constexpr size_t kCounterBytes = 64 * 1024;
-constexpr int64_t kMaxTiles = kCounterBytes / 4;  // n <= 262144 rows per call
+constexpr int64_t kMaxTiles = kCounterBytes / 4 - 1;  // the last slot holds the status word
 
 DmmaWs dmma_ws_layout(int64_t n_total, int32_t k, int mc) {
   const int64_t tiles = (n_total + 15) / 16;
@@ -200,6 +203,136 @@ void dmma_single(DmmaParams& p, const tq_weight_t* w) {
   p.k = w->k;
 }
 
+// ---- tcgen05 GEMM configuration -------------------------------------------------
+
+constexpr int kUmmaMinM = 64;        // from this many tokens on the decoded GEMM uses tcgen05
+constexpr int kSplitTarget = 148;    // split k until about one CTA per SM (B200 SM count)
+constexpr int kStatusOff = (int)kCounterBytes - 4;  // error word: last 4 bytes of the counter region
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+int get_encode_tiled() {
+  if (g_encode_tiled) return TQ_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  TQ_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+  if (q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(cudaErrorNotSupported);
+  g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return TQ_OK;
+}
+
+int umma_bn_for(int32_t m) { return m <= 64 ? 64 : (m <= 128 ? 128 : 256); }
+
+struct UmmaShape {
+  int bn, row_tiles, tok_tiles, splits;
+  size_t partial_bytes;
+};
+
+UmmaShape umma_shape(int64_t n_total, int32_t k, int32_t m) {
+  UmmaShape u;
+  u.bn = umma_bn_for(m);
+  u.row_tiles = (int)((n_total + tq::UM_BM - 1) / tq::UM_BM);
+  u.tok_tiles = (m + u.bn - 1) / u.bn;
+  const int tiles = u.row_tiles * u.tok_tiles;
+  const int blocks = k / 256;
+  int sp = kSplitTarget / tiles;
+  if (sp < 1) sp = 1;
+  if (sp > blocks) sp = blocks;
+  u.splits = sp;
+  u.partial_bytes = sp > 1 ? (size_t)tiles * sp * u.bn * tq::UM_BM * sizeof(float) : 0;
+  return u;
+}
+
+size_t umma_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
+  return kCounterBytes + umma_shape(n_total, k, m).partial_bytes;
+}
+
+// Segments must start on 128-row boundaries for the tile -> segment lookup.
+bool umma_ok(int32_t m, const int32_t* rows, int nseg) {
+  if (m < kUmmaMinM) return false;
+  for (int i = 0; i + 1 < nseg; ++i)
+    if (rows[i] % tq::UM_BM != 0) return false;
+  return true;
+}
+
+int encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw) {
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_in, box_out};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode_tiled(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return TQ_OK;
+}
+
+template <int BN>
+int umma_launch_t(tq::UmmaParams& p, int grid, cudaStream_t stream) {
+  auto kern = tq::umma_kernel<BN>;
+  const size_t smem = tq::UmmaSmem<BN>::ALLOC;
+  static int configured[kMaxDevices];
+  int dev = 0;
+  TQ_CUDA(cudaGetDevice(&dev));
+  if (!configured[dev]) {
+    TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    configured[dev] = 1;
+  }
+  return launch(kern, dim3((unsigned)grid), dim3(tq::UM_THREADS), smem, stream, p);
+}
+
+// y (and handoff) for m tokens of a weight made of `nseg` row segments sharing
+// k and the codebook.  x_f16: device fp16 [m][k].
+int umma_run(const uint8_t* const* codes, const uint16_t* const* scales, const int32_t* rows, int nseg,
+             const uint16_t* codebook, int32_t k, int32_t m, const uint16_t* x_f16, float* y, uint16_t* handoff,
+             float alpha, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int st = get_encode_tiled();
+  if (st != TQ_OK) return st;
+  int64_t n_total = 0;
+  for (int i = 0; i < nseg; ++i) n_total += rows[i];
+  const UmmaShape u = umma_shape(n_total, k, m);
+  if ((int64_t)u.row_tiles * u.tok_tiles > kMaxTiles - 1) return TQ_ERR_SHAPE;
+  if (ws_bytes < kCounterBytes + u.partial_bytes) return TQ_ERR_WORKSPACE;
+  tq::UmmaParams p;
+  memset(&p, 0, sizeof(p));
+  st = encode_2d(&p.tmap_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x_f16, (uint64_t)k, (uint64_t)m, (uint64_t)k * 2,
+                 tq::UM_BK, (uint32_t)u.bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != TQ_OK) return st;
+  int32_t row0 = 0;
+  for (int i = 0; i < nseg; ++i) {
+    st = encode_2d(&p.tmap_codes[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, codes[i], (uint64_t)k / 4, (uint64_t)rows[i],
+                   (uint64_t)k / 4, 16, tq::UM_BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != TQ_OK) return st;
+    p.scales[i] = scales[i];
+    p.seg_row0[i] = row0;
+    p.seg_rows[i] = rows[i];
+    row0 += rows[i];
+  }
+  p.nseg = nseg;
+  p.codebook = codebook;
+  p.n_total = (int32_t)n_total;
+  p.k = k;
+  p.m = m;
+  p.y = y;
+  p.handoff = handoff;
+  p.handoff_rows = handoff ? rows[0] : 0;
+  p.alpha = alpha;
+  p.counters = static_cast<int32_t*>(ws);
+  p.status = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + kStatusOff);
+  p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  p.row_tiles = u.row_tiles;
+  p.tok_tiles = u.tok_tiles;
+  p.splits = u.splits;
+  p.spin_limit = 1u << 21;  // try_wait polls; far above any healthy wait
+  const int grid = u.row_tiles * u.tok_tiles * u.splits;
+  switch (u.bn) {
+    case 64: return umma_launch_t<64>(p, grid, stream);
+    case 128: return umma_launch_t<128>(p, grid, stream);
+    default: return umma_launch_t<256>(p, grid, stream);
+  }
+}
+
 // ---- layer stack helpers -------------------------------------------------------
 
 const double kScaleLo = 0.005, kScaleHi = 0.03;
@@ -237,11 +370,20 @@ int phase_check(const tq_layer_t* L, int phase, int* nops, const tq_weight_t* op
 }
 
 // Workspace of one phase call at m tokens:
-//  [dmma counters + partials][x' fp16 [m][k] when m > 1]
-size_t phase_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
+//  [counters | partial sums (largest kernel choice)][x' fp16 [m][k] when m > 1]
+size_t matmul_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
   const int mc = (m <= 1) ? 1 : dmma_nt_for(m < kDmmaMaxM ? m : kDmmaMaxM) * 8;
   size_t b = dmma_ws_layout(n_total, k, mc).bytes;
-  if (m > 1) b = round_up(b, 256) + round_up((size_t)m * k * 2, 256);
+  if (m >= kUmmaMinM) {
+    const size_t u = umma_ws_bytes(n_total, k, m);
+    if (u > b) b = u;
+  }
+  return round_up(b, 256);
+}
+
+size_t phase_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
+  size_t b = matmul_ws_bytes(n_total, k, m);
+  if (m > 1) b += round_up((size_t)m * k * 2, 256);
   return b;
 }
 
@@ -278,9 +420,9 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
     p.rht_seed = seed;
     return dmma_run(p, true, ws, ws_bytes, num_sms, stream);
   }
-  // m > 1: RHT to fp16 in the workspace tail, then the small-batch kernel in
-  // chunks of up to 64 tokens.
-  const size_t dm_bytes = round_up(dmma_ws_layout(n_total, k, dmma_nt_for(m < kDmmaMaxM ? m : kDmmaMaxM) * 8).bytes, 256);
+  // m > 1: RHT to fp16 in the workspace tail, then the tcgen05 GEMM (m >= 64)
+  // or the small-batch kernel in chunks of up to 64 tokens.
+  const size_t dm_bytes = matmul_ws_bytes(n_total, k, m);
   uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + dm_bytes);
   {
     const int64_t tasks = (int64_t)m * (k / 512);
@@ -290,6 +432,16 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
                 (void*)xr);
     if (st != TQ_OK) return st;
   }
+  int32_t rows[3];
+  const uint8_t* cptr[3];
+  const uint16_t* sptr[3];
+  for (int i = 0; i < nops; ++i) {
+    rows[i] = ops[i]->n;
+    cptr[i] = ops[i]->codes_d;
+    sptr[i] = ops[i]->scales_d;
+  }
+  if (umma_ok(m, rows, nops))
+    return umma_run(cptr, sptr, rows, nops, ops[0]->codebook_d, k, m, xr, y, handoff, p.alpha, ws, dm_bytes, stream);
   for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
     DmmaParams pc = p;
     pc.m = (m - t0) < kDmmaMaxM ? (m - t0) : kDmmaMaxM;
@@ -300,14 +452,6 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
     if (st != TQ_OK) return st;
   }
   return TQ_OK;
-}
-
-int64_t phase_n(const tq_layer_t* L, int phase) {
-  const tq_weight_t* ops[3];
-  int n = phase_ops(L, phase, ops);
-  int64_t t = 0;
-  for (int i = 0; i < n; ++i) t += ops[i]->n;
-  return t;
 }
 
 }  // namespace
@@ -393,8 +537,7 @@ int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* worksp
 int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes) {
   if (!bytes) return TQ_ERR_NULL;
   if (n < 1 || !k_ok(k) || m < 0 || m > 4096) return TQ_ERR_SHAPE;
-  const int mm = m < 1 ? 1 : (m < kDmmaMaxM ? m : kDmmaMaxM);
-  *bytes = dmma_ws_layout(n, k, dmma_nt_for(mm) * 8).bytes;
+  *bytes = matmul_ws_bytes(n, k, m < 1 ? 1 : m);
   return TQ_OK;
 }
 
@@ -409,6 +552,13 @@ int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float*
   int sms = 0;
   st = check_arch(&sms);
   if (st != TQ_OK) return st;
+  if (m >= kUmmaMinM) {
+    const uint8_t* c = w->codes_d;
+    const uint16_t* sc = w->scales_d;
+    const int32_t rows = w->n;
+    return umma_run(&c, &sc, &rows, 1, w->codebook_d, w->k, m, x_rot_f16_d, y_d, nullptr, 0.f, workspace_d, ws_bytes,
+                    (cudaStream_t)stream);
+  }
   for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
     DmmaParams p;
     dmma_single(p, w);
@@ -597,7 +747,7 @@ const char* tq_status_string(int status) {
     case TQ_ERR_WORKSPACE: return "workspace missing or too small";
     case TQ_ERR_CUDA: return "CUDA runtime error (see tq_last_cuda_error)";
     case TQ_ERR_TIMEOUT: return "bounded device wait expired";
-    case TQ_ERR_SCRATCH: return "problem larger than the built-in scratch of tq_gemv_noalloc (n > 262144)";
+    case TQ_ERR_SCRATCH: return "problem larger than the built-in scratch of tq_gemv_noalloc (n > 262128)";
     default: return "unknown status";
   }
 }

@@ -132,7 +132,7 @@ TQ_API int tq_gemv_workspace(int32_t n, int32_t k, size_t* bytes);
  * before the first call (tq_workspace_init); every call of this library leaves
  * it zero again, so one workspace may serve calls of any shape in turn.  The
  * rest is scratch.  Calls that share a workspace must not overlap on the GPU.
- * n is limited to 262144 rows per call (TQ_ERR_SHAPE). */
+ * n is limited to 262128 rows per call (TQ_ERR_SHAPE). */
 TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* workspace_d, size_t ws_bytes,
             void* stream);
 
@@ -152,7 +152,7 @@ TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void*
  * the array, which keeps the last call's contents: calls that overlap on the
  * GPU (for example on two streams) race and give wrong results, so run them
  * one after another.
- * Limit: n <= 262144 rows (TQ_ERR_SCRATCH beyond it); k any positive
+ * Limit: n <= 262128 rows (TQ_ERR_SCRATCH beyond it); k any positive
  * multiple of 512. */
 #define TQ_GEMV_NOALLOC_SCRATCH_BYTES ((size_t)(1u << 20) + (size_t)(64u << 10))
 TQ_API int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* stream);

@@ -1,0 +1,42 @@
+"""The decode-to-shared-memory tcgen05 GEMM (tq_gemm at m >= 64) against the
+oracle: tile shapes with split-k, ragged rows and several token tiles."""
+import numpy as np
+import pytest
+
+import oracle
+import tqsynth
+from gpu_util import TOL, dev_weight, f16_exact, host_weight, oracle_linear
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(n, k, m, rows=None, seed=2):
+    import torch
+
+    import decode_matmul_b200 as tq
+    hw = host_weight(seed, 0, 5, n, k)
+    x = tqsynth.activations(seed, m, k)
+    xr = f16_exact(oracle.rht(x, m, k, 11))
+    xd = torch.from_numpy(xr.astype(np.float16)).cuda()
+    y = tq.tq_gemm(dev_weight(hw), xd).cpu().numpy()
+    if rows is None:
+        want = oracle_linear(hw, xr, m)
+        return oracle.rel_err(y, want)
+    errs = []
+    for r0, r1 in rows:
+        want = oracle.linear_rows(hw.codes, hw.scales, hw.codebook, k, xr, m, r0, r1)
+        errs.append(oracle.rel_err(y[:, r0:r1], want))
+    return max(errs)
+
+
+@pytest.mark.parametrize("n,k,m", [(128, 512, 64), (1040, 1536, 64), (640, 2560, 128), (384, 1024, 200),
+                                   (256, 512, 512)])
+def test_tcgen05_gemm_full_compare(n, k, m):
+    err = _run(n, k, m)
+    assert err < TOL, err
+
+
+def test_tcgen05_gemm_split_k_large_k():
+    # 20 row tiles x 1 token tile -> split k across the blocks of k = 9728
+    err = _run(2560, 9728, 64, rows=[(0, 8), (1277, 1283), (2552, 2560)])
+    assert err < TOL, err
