@@ -9,6 +9,7 @@
 #include "tq_decode.cuh"
 #include "tq_dmma.cuh"
 #include "tq_rht.cuh"
+#include "tq_stack1.cuh"
 #include "tq_umma.cuh"
 
 #include <cudaTypedefs.h>
@@ -614,9 +615,11 @@ int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf1
 }
 
 // Stack workspace: [phase workspace][y fp32 [m][max n]][a bf16 [m][q]]
-// [b bf16 [m][hidden]][c bf16 [m][inter]][h bf16 [m][hidden]]
+// [b bf16 [m][hidden]][c bf16 [m][inter]][h bf16 [m][hidden]][RHT sign bits]
+// [barrier word]
 struct StackWs {
-  size_t phase, y, a, b, c, h, total;
+  size_t phase, y, a, b, c, h, signs, sync, total;
+  uint32_t sign_words;
 };
 
 static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, StackWs* L) {
@@ -645,13 +648,107 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
     if (L0.gate.n > cmax) cmax = L0.gate.n;
     if (L0.down.n > hmax) hmax = L0.down.n;
   }
+  // at batch 1 the persistent stack kernel keeps two partial-sum slots for
+  // every warp it may run (at most DMMA_MAX_WARPS)
+  if (m == 1) {
+    const size_t pk = kCounterBytes + (size_t)tq::DMMA_MAX_WARPS * 2 * 16 * sizeof(float);
+    if (phase < pk) phase = pk;
+  }
+  uint64_t words = 0;
+  for (int l = 0; l < n_layers; ++l)
+    words += ((uint64_t)layers[l].q.k + layers[l].o.k + layers[l].gate.k + layers[l].down.k) / 32;
   L->phase = 0;
   L->y = round_up(phase, 256);
   L->a = L->y + round_up((size_t)m * ymax * 4, 256);
   L->b = L->a + round_up((size_t)m * amax * 2, 256);
   L->c = L->b + round_up((size_t)m * bmax * 2, 256);
   L->h = L->c + round_up((size_t)m * cmax * 2, 256);
-  L->total = L->h + round_up((size_t)m * hmax * 2, 256);
+  L->signs = L->h + round_up((size_t)m * hmax * 2, 256);
+  L->sign_words = (uint32_t)words;
+  L->sync = L->signs + round_up((size_t)words * 4, 256);
+  L->total = L->sync + 256;
+  return TQ_OK;
+}
+
+// The whole batch-1 stack as one cooperative persistent kernel.  Returns
+// TQ_ERR_SHAPE (and launches nothing) when the stack does not qualify: more
+// than STACK_MAX_LAYERS layers, phases with different codebooks, or a phase
+// too wide for shared memory.
+static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in, uint64_t seed,
+                      uint16_t* h_out, char* ws, const StackWs& L, int sms, cudaStream_t s) {
+  if (n_layers > tq::STACK_MAX_LAYERS) return TQ_ERR_SHAPE;
+  static thread_local tq::StackParams sp;  // large (~25 KB): per-thread storage, copied into the launch
+  memset(&sp, 0, sizeof(sp));
+  const uint16_t* cb = layers[0].q.codebook_d;
+  int32_t kmax = 0;
+  uint32_t off = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    const tq_layer_t& ly = layers[l];
+    const tq_weight_t* ops[7] = {&ly.q, &ly.k, &ly.v, &ly.o, &ly.gate, &ly.up, &ly.down};
+    tq::StackLayerDev& d = sp.layers[l];
+    for (int i = 0; i < 7; ++i) {
+      if (ops[i]->codebook_d != cb) return TQ_ERR_SHAPE;
+      d.codes[i] = ops[i]->codes_d;
+      d.scales[i] = ops[i]->scales_d;
+      d.n[i] = ops[i]->n;
+    }
+    const int32_t ks[4] = {ly.q.k, ly.o.k, ly.gate.k, ly.down.k};
+    const int32_t nt[4] = {ly.q.n + ly.k.n + ly.v.n, ly.o.n, ly.gate.n + ly.up.n, ly.down.n};
+    for (int ph = 0; ph < 4; ++ph) {
+      d.k[ph] = ks[ph];
+      d.sign_off[ph] = off;
+      off += (uint32_t)ks[ph] / 32;
+      d.alpha[ph] = stack_alpha(ks[ph]);
+      if (ks[ph] > kmax) kmax = ks[ph];
+      if ((nt[ph] + 15) / 16 > kMaxTiles) return TQ_ERR_SHAPE;
+    }
+  }
+  const int lv = dmma_lv_for(true, kmax);
+  const size_t smem = (16384u << lv) + (size_t)kmax * 4 + sizeof(tq::DmmaParams) + 16;
+  if (smem > 227 * 1024) return TQ_ERR_SHAPE;
+  sp.n_layers = n_layers;
+  sp.lv = lv;
+  sp.codebook = cb;
+  sp.h_in = h_in;
+  sp.h_out = h_out;
+  sp.buf[0] = reinterpret_cast<uint16_t*>(ws + L.a);
+  sp.buf[1] = reinterpret_cast<uint16_t*>(ws + L.b);
+  sp.buf[2] = reinterpret_cast<uint16_t*>(ws + L.c);
+  sp.buf[3] = reinterpret_cast<uint16_t*>(ws + L.h);
+  sp.y = reinterpret_cast<float*>(ws + L.y);
+  sp.signs = reinterpret_cast<uint32_t*>(ws + L.signs);
+  sp.sign_words = L.sign_words;
+  sp.seed = seed;
+  sp.counters = reinterpret_cast<int32_t*>(ws);
+  sp.status = reinterpret_cast<int32_t*>(ws + kStatusOff);
+  sp.partials = reinterpret_cast<float*>(ws + kCounterBytes);
+  sp.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
+  sp.spin_limit = 1u << 24;  // x 64 ns sleeps: ~1 s, far above any healthy phase
+  void (*kern)(tq::StackParams);
+  switch (lv) {
+    case 3: kern = tq::stack1_kernel<3>; break;
+    case 2: kern = tq::stack1_kernel<2>; break;
+    case 1: kern = tq::stack1_kernel<1>; break;
+    default: kern = tq::stack1_kernel<0>; break;
+  }
+  TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+  int occ = 0;
+  TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
+  if (occ < 1) return TQ_ERR_SHAPE;
+  // partial sums: every warp of the grid may hold two tile partials
+  if ((size_t)sms * tq::DMMA_WARPS * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
+  TQ_CUDA(cudaMemsetAsync(ws + L.sync, 0, 256, s));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)sms);
+  cfg.blockDim = dim3(tq::DMMA_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  TQ_CUDA(cudaLaunchKernelEx(&cfg, kern, sp));
   return TQ_OK;
 }
 
@@ -684,6 +781,10 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
   const size_t phase_bytes = L.y;
   cudaStream_t s = (cudaStream_t)stream;
+  if (m == 1) {
+    st = stack1_run(layers, n_layers, h_in_bf16_d, seed, h_out_bf16_d, ws, L, sms, s);
+    if (st != TQ_ERR_SHAPE) return st;  // TQ_ERR_SHAPE: not eligible, run phase by phase
+  }
   for (int l = 0; l < n_layers; ++l) {
     const uint16_t* in0 = (l == 0) ? h_in_bf16_d : h;
     uint16_t* out3 = (l == n_layers - 1) ? h_out_bf16_d : h;

@@ -273,22 +273,15 @@ __device__ __forceinline__ void dmma_flush(const DmmaParams& p, int64_t W, int64
   if (lane == 0) p.counters[t] = 0;  // leave the counter ready for the next call
 }
 
-// LV = log2(number of codebook views); NT = number of 8-token MMA column
-// tiles (small batch); HILO = batch-1 mode with fp32 x' split in hi/lo.
-template <int LV, int NT, bool HILO>
-__global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_constant__ DmmaParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+// Replicate the codebook into V = 2^LV shared-memory views (entry e of view
+// v at byte e*8V + 8v).
+template <int LV>
+__device__ __forceinline__ void build_views(uint8_t* smem, const uint16_t* __restrict__ codebook, int tid,
+                                            int nthreads) {
   constexpr int V = 1 << LV;
   constexpr int SH = 3 + LV;
-  uint8_t* xs = smem + (16384 << LV);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, q = lane & 3;
-
-  pdl_launch_dependents();
-
-  // Codebook views (no kernel in the stream writes the codebook).
-  for (int e = tid; e < 2048; e += DMMA_THREADS) {
-    const uint2 ent = reinterpret_cast<const uint2*>(p.codebook)[e];
+  for (int e = tid; e < 2048; e += nthreads) {
+    const uint2 ent = reinterpret_cast<const uint2*>(codebook)[e];
     uint8_t* dst = smem + (e << SH);
     if (V == 1) {
       *reinterpret_cast<uint2*>(dst) = ent;
@@ -298,45 +291,54 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
         *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(ent.x, ent.y, ent.x, ent.y);
     }
   }
+}
 
-  const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
-  const bool active = W < p.active_warps;
-  const int64_t wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
-  const int64_t we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
-
-  // The weights are not written by any kernel of the stream: prefetch the
-  // first chunk before waiting on the previous kernel.
-  int t = 0, b = 0;  // tile and block of the current unit (no divisions in the loop)
+// Units [wb, we) of global warp W, the tile/block it starts at and its first
+// chunk of code bytes (loaded ahead: the weights never depend on activations).
+struct DmmaCursor {
+  int64_t wb, we;
+  int t, b;
   DmmaRows rows;
   DmmaChunk cur;
-  if (wb < we) {
-    t = (int)(wb / p.blocks);
-    b = (int)(wb - (int64_t)t * p.blocks);
-    rows = dmma_rows(p, t, g, q);
-    cur = dmma_fetch(rows, b);
+};
+
+__device__ __forceinline__ void dmma_begin(const DmmaParams& p, int64_t W, int g, int q, DmmaCursor& c) {
+  const bool active = W < p.active_warps;
+  c.wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
+  c.we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
+  c.t = c.b = 0;
+  if (c.wb < c.we) {
+    c.t = (int)(c.wb / p.blocks);
+    c.b = (int)(c.wb - (int64_t)c.t * p.blocks);
+    c.rows = dmma_rows(p, c.t, g, q);
+    c.cur = dmma_fetch(c.rows, c.b);
   }
+}
 
-  pdl_wait();
+// Batch-1 activation quad of one MMA step for lanes 0-7 (lanes g = 0 / 1 hold
+// the hi / lo column); the other lanes own MMA columns that are never read
+// and skip the load (predicated, no branch).
+__device__ __forceinline__ uint2 lds_b_hilo(const uint8_t* addr, int lane) {
+  uint2 v = make_uint2(0u, 0u);
+  asm volatile(
+      "{\n .reg .pred p;\n setp.lt.u32 p, %2, 8;\n @p ld.shared.v2.u32 {%0,%1}, [%3];\n}\n"
+      : "+r"(v.x), "+r"(v.y)
+      : "r"(lane), "r"(smem_u32(addr)));
+  return v;
+}
 
-  if (HILO) {
-    if (p.x_bf16) {
-      for (int blk = warp; blk < p.k / 512; blk += DMMA_WARPS) {
-        float v[16];
-        rht512_warp(p.x_bf16, blk, p.rht_seed, v);
-#pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4)
-          store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
-      }
-    } else {
-      for (int G = tid; G < (p.k >> 2); G += DMMA_THREADS) {
-        const float4 x = reinterpret_cast<const float4*>(p.x_f32)[G];
-        store_hilo(xs, G, x.x, x.y, x.z, x.w);
-      }
-    }
-  }
-  __syncthreads();
-  if (wb >= we) return;
-
+// The unit loop of one warp: decode its units, run the MMAs, flush tiles.
+// `smem` holds the codebook views, `xs` the batch-1 activations (hi/lo).
+template <int LV, int NT, bool HILO>
+__device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* smem, const uint8_t* xs, int64_t W,
+                                           DmmaCursor& c, int lane) {
+  constexpr int V = 1 << LV;
+  constexpr int SH = 3 + LV;
+  const int g = lane >> 2, q = lane & 3;
+  if (c.wb >= c.we) return;
+  int t = c.t, b = c.b;
+  DmmaRows rows = c.rows;
+  DmmaChunk cur = c.cur;
   const uint32_t vofs = (uint32_t)((lane & (V - 1)) << 3);
   // two accumulator sets (even / odd code steps) halve the MMA dependency chain
   float acc[NT][4], acc2[NT][4];
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
 
-  const int nunits = (int)(we - wb);
+  const int nunits = (int)(c.we - c.wb);
   for (int iu = 0; iu < nunits; ++iu) {
     int tn = t, bn = b + 1;
     if (bn == p.blocks) {
@@ -391,10 +393,9 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
         a[1] = hmul2_u32(eb.x, sb2);
         a[3] = hmul2_u32(eb.y, sb2);
         // B columns other than the live ones (hi/lo at batch 1, tokens < m
-        // otherwise) only feed C columns that are never read, so every lane
-        // loads a valid activation quad without predicates.
+        // otherwise) only feed C columns that are never read.
         if (HILO) {
-          const uint2 bw = *reinterpret_cast<const uint2*>(xs_lane + j * 64);
+          const uint2 bw = lds_b_hilo(xs_lane + j * 64, lane);
           mma_16816((j & 1) ? acc2[0] : acc[0], a, bw.x, bw.y);
         } else {
 #pragma unroll
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
       for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[jt][i] += acc2[jt][i];
-      dmma_flush<NT, HILO>(p, W, wb, we, t, g, q, acc);
+      dmma_flush<NT, HILO>(p, W, c.wb, c.we, t, g, q, acc);
 #pragma unroll
       for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
@@ -422,6 +423,45 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
     rows = nrows;
     cur = nxt;
   }
+}
+
+// Batch-1 activations of the block: x' = RHT(x_bf16) computed here, or x' fp32
+// given, split into hi/lo fp16 quads in shared memory.
+__device__ __forceinline__ void dmma_prologue_hilo(const DmmaParams& p, uint8_t* xs, int tid, int nthreads) {
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nthreads >> 5;
+  if (p.x_bf16) {
+    for (int blk = warp; blk < p.k / 512; blk += nwarps) {
+      float v[16];
+      rht512_warp(p.x_bf16, blk, p.rht_seed, v);
+#pragma unroll
+      for (int r4 = 0; r4 < 4; ++r4)
+        store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
+    }
+  } else {
+    for (int G = tid; G < (p.k >> 2); G += nthreads) {
+      const float4 x = reinterpret_cast<const float4*>(p.x_f32)[G];
+      store_hilo(xs, G, x.x, x.y, x.z, x.w);
+    }
+  }
+}
+
+// LV = log2(number of codebook views); NT = number of 8-token MMA column
+// tiles (small batch); HILO = batch-1 mode with fp32 x' split in hi/lo.
+template <int LV, int NT, bool HILO>
+__global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_constant__ DmmaParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* xs = smem + (16384 << LV);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  pdl_launch_dependents();
+  build_views<LV>(smem, p.codebook, tid, DMMA_THREADS);  // no kernel of the stream writes the codebook
+  const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
+  DmmaCursor c;
+  dmma_begin(p, W, lane >> 2, lane & 3, c);  // weights: prefetched before waiting on the previous kernel
+  pdl_wait();
+  if (HILO) dmma_prologue_hilo(p, xs, tid, DMMA_THREADS);
+  __syncthreads();
+  dmma_units<LV, NT, HILO>(p, smem, xs, W, c, lane);
 }
 
 }  // namespace tq
