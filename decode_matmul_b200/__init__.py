@@ -23,7 +23,8 @@ OPS = ("q", "k", "v", "o", "gate", "up", "down")
 
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
-           "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc")
+           "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
+           "tq_layer_stack_buffers")
 
 
 class TqError(RuntimeError):
@@ -79,6 +80,7 @@ def _lib():
             "tq_layer_stack_workspace": ([LY, i32, i32, szp], ctypes.c_int),
             "tq_layer_phase": ([LY, i32, vp, i32, u64, vp, vp, vp, sz, vp], ctypes.c_int),
             "tq_layer_stack": ([LY, i32, vp, i32, u64, vp, vp, sz, vp], ctypes.c_int),
+            "tq_layer_stack_buffers": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "tq_last_cuda_error": ([], ctypes.c_int),
         }
@@ -236,6 +238,15 @@ def tq_layer_phase(layer: tq_layer_t, phase: int, x_bf16, phase_seed: int, y, ha
     m = x_bf16.shape[0]
     _ok(_lib().tq_layer_phase(ctypes.byref(layer), phase, _ptr(x_bf16), m, phase_seed, _ptr(y), _ptr(handoff),
                               _ptr(ws), ws.numel(), _stream(stream)), "tq_layer_phase")
+
+
+def tq_layer_stack_buffers(layers, m: int):
+    """Workspace byte offsets of the last layer's q, o, gate handoffs, its
+    input h and the last phase's fp32 y."""
+    arr = (tq_layer_t * len(layers))(*layers)
+    out = (ctypes.c_size_t * 5)()
+    _ok(_lib().tq_layer_stack_buffers(arr, len(layers), m, out), "tq_layer_stack_buffers")
+    return list(out)
 
 
 class StackArgs:

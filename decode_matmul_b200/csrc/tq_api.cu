@@ -752,6 +752,19 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   return TQ_OK;
 }
 
+int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[5]) {
+  if (!offsets) return TQ_ERR_NULL;
+  StackWs L;
+  int st = stack_layout(layers, n_layers, m, &L);
+  if (st != TQ_OK) return st;
+  offsets[0] = L.a;
+  offsets[1] = L.b;
+  offsets[2] = L.c;
+  offsets[3] = L.h;
+  offsets[4] = L.y;
+  return TQ_OK;
+}
+
 int tq_layer_stack_workspace(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t* bytes) {
   if (!bytes) return TQ_ERR_NULL;
   StackWs L;

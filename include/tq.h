@@ -216,6 +216,16 @@ TQ_API int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t
 TQ_API int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m, uint64_t seed,
                    uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes, void* stream);
 
+/* Byte offsets, inside a tq_layer_stack workspace for these layers and m,
+ * of the bf16 buffers that hold the last layer's phase handoffs when
+ * tq_layer_stack has returned: offsets[0] = q handoff [m][q.n], offsets[1] =
+ * o handoff [m][o.n], offsets[2] = gate handoff [m][gate.n], offsets[3] = the
+ * last layer's input h [m][hidden] (for n_layers >= 2; with one layer the
+ * input is h_in); offsets[4] = fp32 y of the last phase (down) [m][down.n].
+ * The last phase's handoff is h_out itself.  For inspection and tests; the
+ * buffers are scratch for the next call. */
+TQ_API int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[5]);
+
 /* Human-readable text of a status code (static storage). */
 TQ_API const char* tq_status_string(int status);
 
