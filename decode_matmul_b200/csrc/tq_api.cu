@@ -425,14 +425,6 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
   // or the small-batch kernel in chunks of up to 64 tokens.
   const size_t dm_bytes = matmul_ws_bytes(n_total, k, m);
   uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + dm_bytes);
-  {
-    const int64_t tasks = (int64_t)m * (k / 512);
-    int64_t blocks = (tasks + 7) / 8;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    st = launch(tq::rht_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, stream, x, (int)m, (int)k, seed,
-                (void*)xr);
-    if (st != TQ_OK) return st;
-  }
   int32_t rows[3];
   const uint8_t* cptr[3];
   const uint16_t* sptr[3];
@@ -441,7 +433,18 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
     cptr[i] = ops[i]->codes_d;
     sptr[i] = ops[i]->scales_d;
   }
-  if (umma_ok(m, rows, nops))
+  const bool use_umma = umma_ok(m, rows, nops);
+  {
+    // x' fp16: row-major for the TMA of the tcgen05 GEMM, fragment order for
+    // the small-batch kernel
+    const int64_t tasks = (int64_t)m * (k / 512);
+    int64_t blocks = (tasks + 7) / 8;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    st = launch(use_umma ? tq::rht_kernel<1> : tq::rht_kernel<2>, dim3((unsigned)blocks), dim3(256), 0, stream, x,
+                (int)m, (int)k, seed, (void*)xr);
+    if (st != TQ_OK) return st;
+  }
+  if (use_umma)
     return umma_run(cptr, sptr, rows, nops, ops[0]->codebook_d, k, m, xr, y, handoff, p.alpha, ws, dm_bytes, stream);
   for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
     DmmaParams pc = p;
@@ -505,9 +508,9 @@ int tq_rht(const uint16_t* x_bf16_d, int32_t m, int32_t k, uint64_t seed, void* 
   int64_t blocks = (tasks + 7) / 8;
   if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
   if (out_dtype == TQ_F16)
-    return launch(tq::rht_kernel<true>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+    return launch(tq::rht_kernel<1>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
                   (int)k, seed, x_rot_d);
-  return launch(tq::rht_kernel<false>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+  return launch(tq::rht_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
                 (int)k, seed, x_rot_d);
 }
 
@@ -539,6 +542,7 @@ int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes) {
   if (!bytes) return TQ_ERR_NULL;
   if (n < 1 || !k_ok(k) || m < 0 || m > 4096) return TQ_ERR_SHAPE;
   *bytes = matmul_ws_bytes(n, k, m < 1 ? 1 : m);
+  if (m > 1 && m < kUmmaMinM) *bytes += round_up((size_t)m * k * 2, 256);  // x' in fragment order
   return TQ_OK;
 }
 
@@ -560,11 +564,24 @@ int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float*
     return umma_run(&c, &sc, &rows, 1, w->codebook_d, w->k, m, x_rot_f16_d, y_d, nullptr, 0.f, workspace_d, ws_bytes,
                     (cudaStream_t)stream);
   }
+  // the small-batch kernel reads x' in fragment order: permute it into the
+  // workspace after the matmul scratch
+  const size_t mm_bytes = matmul_ws_bytes(w->n, w->k, m);
+  if (ws_bytes < mm_bytes + (size_t)m * w->k * 2) return TQ_ERR_WORKSPACE;
+  uint16_t* xp = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace_d) + mm_bytes);
+  {
+    const int64_t groups = (int64_t)m * (w->k / 4);
+    int64_t blocks = (groups + 255) / 256;
+    if (blocks > (int64_t)sms * 16) blocks = (int64_t)sms * 16;
+    st = launch(tq::frag_permute_kernel, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_rot_f16_d,
+                (int)m, (int)w->k, xp);
+    if (st != TQ_OK) return st;
+  }
   for (int32_t t0 = 0; t0 < m; t0 += kDmmaMaxM) {
     DmmaParams p;
     dmma_single(p, w);
     p.m = (m - t0) < kDmmaMaxM ? (m - t0) : kDmmaMaxM;
-    p.x_f16 = x_rot_f16_d + (size_t)t0 * w->k;
+    p.x_f16 = xp + (size_t)t0 * w->k;
     p.y = y_d + (size_t)t0 * w->n;
     st = dmma_run(p, false, workspace_d, ws_bytes, sms, (cudaStream_t)stream);
     if (st != TQ_OK) return st;

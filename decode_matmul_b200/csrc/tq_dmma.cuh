@@ -55,7 +55,7 @@ struct DmmaParams {
   const float* x_f32;      // batch 1: x' fp32 [k]
   const uint16_t* x_bf16;  // batch 1, fused RHT: x bf16 [k]
   uint64_t rht_seed;
-  const uint16_t* x_f16;   // small batch: x' fp16 [m][k]
+  const uint16_t* x_f16;   // small batch: x' fp16 [m][k] in fragment order (frag_pos)
   float* y;                // [m][n_total] or null
   uint16_t* handoff;       // [m][handoff_rows] bf16 or null
   int32_t handoff_rows;
@@ -365,7 +365,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
     const uint16_t* xg_lane[NT];
 #pragma unroll
     for (int jt = 0; jt < NT; ++jt)
-      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + 4 * (size_t)(b * 64 + q * 16);
+      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + (size_t)b * 256 + q * 4;
     // previous code byte of each row chunk (state of code 0); 0 at a block start
     uint32_t pa = __shfl_up_sync(0xffffffffu, cur.ca.w, 1) >> 24;
     uint32_t pb = __shfl_up_sync(0xffffffffu, cur.cb.w, 1) >> 24;
@@ -400,7 +400,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
         } else {
 #pragma unroll
           for (int jt = 0; jt < NT; ++jt) {
-            const uint2 bv = __ldg(reinterpret_cast<const uint2*>(xg_lane[jt] + 4 * j));
+            const uint2 bv = __ldg(reinterpret_cast<const uint2*>(xg_lane[jt] + 16 * j));
             mma_16816((j & 1) ? acc2[jt] : acc[jt], a, bv.x, bv.y);
           }
         }

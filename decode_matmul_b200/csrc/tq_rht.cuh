@@ -66,8 +66,18 @@ __device__ __forceinline__ void rht512_warp(const uint16_t* __restrict__ x_row, 
   for (int r = 0; r < 16; ++r) v[r] *= inv;
 }
 
-// Standalone RHT: grid-stride over (row, block) warp tasks.
-template <bool OUT_F16>
+// Position of element k of a row in "fragment order": inside each 256-weight
+// block the 64 groups of 4 are stored step-major, (j, q) for group 16q + j,
+// so that the four quads one MMA step of the small-batch kernel reads (lanes
+// q = 0..3, step j) are 32 contiguous bytes.
+__host__ __device__ __forceinline__ int frag_pos(int k) {
+  const int b = k >> 8, G = (k & 255) >> 2, e = k & 3;
+  return (b << 8) + ((((G & 15) << 2) + (G >> 4)) << 2) + e;
+}
+
+// Standalone RHT: grid-stride over (row, block) warp tasks.  MODE 0: fp32
+// row-major; 1: fp16 row-major; 2: fp16 in fragment order (frag_pos).
+template <int MODE>
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x, int m, int k, uint64_t seed,
                                                   void* __restrict__ out) {
   pdl_wait();
@@ -82,16 +92,36 @@ __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x
     float v[16];
     rht512_warp(x + (size_t)row * k, blk, seed, v);
     const size_t o = (size_t)row * k + (size_t)blk * 512 + lane * 16;
-    if (OUT_F16) {
+    if (MODE == 1) {
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + o);
       dst[0] = make_uint4(f2_to_h2(v[0], v[1]), f2_to_h2(v[2], v[3]), f2_to_h2(v[4], v[5]), f2_to_h2(v[6], v[7]));
       dst[1] = make_uint4(f2_to_h2(v[8], v[9]), f2_to_h2(v[10], v[11]), f2_to_h2(v[12], v[13]),
                           f2_to_h2(v[14], v[15]));
+    } else if (MODE == 2) {
+      uint16_t* rowp = reinterpret_cast<uint16_t*>(out) + (size_t)row * k;
+#pragma unroll
+      for (int r4 = 0; r4 < 4; ++r4) {
+        const int kk = blk * 512 + lane * 16 + 4 * r4;
+        *reinterpret_cast<uint2*>(rowp + frag_pos(kk)) =
+            make_uint2(f2_to_h2(v[4 * r4], v[4 * r4 + 1]), f2_to_h2(v[4 * r4 + 2], v[4 * r4 + 3]));
+      }
     } else {
       float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + o);
 #pragma unroll
       for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
+  }
+}
+
+// fp16 [m][k] row-major -> fragment order (one thread per group of 4).
+__global__ void __launch_bounds__(256) frag_permute_kernel(const uint16_t* __restrict__ x, int m, int k,
+                                                           uint16_t* __restrict__ out) {
+  const long long groups = (long long)m * (k / 4);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < groups;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / (k / 4);
+    const int kk = (int)(i - row * (k / 4)) * 4;
+    *reinterpret_cast<uint2*>(out + row * k + frag_pos(kk)) = *reinterpret_cast<const uint2*>(x + row * k + kk);
   }
 }
 
