@@ -419,7 +419,7 @@ def main():
                       "unit": "GB/s", "frac": bytes_step_layer / (kern_ms_layer * 1e-3) / 1e9 / hbm,
                       "traffic": None, "peak_source": peak_src,
                       "kernel": "rht_kernel + dmma_kernel (mma.sync register decode), all 4 phases",
-                      "phase_ms": ph_ms, "phase_bytes": pb} if m < 64 else
+                      "phase_ms": ph_ms, "phase_bytes": pb} if m < 32 else
                      {"bound": "tensor", "achieved": tensor_tflops, "peak": tflops, "unit": "TFLOP/s",
                       "frac": tensor_tflops / tflops, "traffic": None, "peak_source": peak_src,
                       "kernel": "rht_kernel + umma_kernel (tcgen05 decode-to-smem GEMM), all 4 phases",
@@ -429,7 +429,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": "tok/s", "h2d_bytes_per_step": int(h_host.numel() * 2),
                 "d2h_bytes_per_step": int(o_host.numel() * 2)},
-        "gpu_launches": args.steps * (1 if m == 1 else 4 * shape.layers * (2 if m >= 64 else 1 + math.ceil(m / 64))),
+        "gpu_launches": args.steps * (1 if m == 1 else 4 * shape.layers * 2),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
