@@ -275,7 +275,8 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
         const int bn = b_lo + (i >> 2) + 1;
         if (bn < b_hi) sc_next = __ldg(srow + bn);
       }
-      if (*abort_flag || !mbar_wait(bar_full + 8 * s, rr & 1, p.spin_limit)) {
+      // the stop decision is warp-uniform: the warp-collective ops below need every lane
+      if (!__all_sync(0xffffffffu, !*abort_flag && mbar_wait(bar_full + 8 * s, rr & 1, p.spin_limit))) {
         *abort_flag = 1;
         break;
       }
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     // always wait for the MMAs issued so far (TMEM is freed below), read only
     // when nothing timed out
     const bool done = mbar_wait(bar_acc, 0, p.spin_limit);
-    const bool ok = done && !*abort_flag;
+    const bool ok = __all_sync(0xffffffffu, done && !*abort_flag);  // tcgen05.ld is warp-collective
     if (!ok) *abort_flag = 1;
     tc_fence_after();
     const int n = row0 + wq * 32 + lane;
