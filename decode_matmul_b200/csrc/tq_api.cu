@@ -633,9 +633,12 @@ int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf1
 
 // Stack workspace: [phase workspace][y fp32 [m][max n]][a bf16 [m][q]]
 // [b bf16 [m][hidden]][c bf16 [m][inter]][h bf16 [m][hidden]][RHT sign bits]
-// [barrier word]
+// [per-phase parameter and straddling-tile tables (batch-1 persistent
+// kernel)][barrier word]
+constexpr int kStackMaxCtas = 256;  // bound on the persistent stack kernel's grid (tables sized by it)
+
 struct StackWs {
-  size_t phase, y, a, b, c, h, signs, sync, total;
+  size_t phase, y, a, b, c, h, signs, params, straddle, sync, total;
   uint32_t sign_words;
 };
 
@@ -676,13 +679,18 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
     words += ((uint64_t)layers[l].q.k + layers[l].o.k + layers[l].gate.k + layers[l].down.k) / 32;
   L->phase = 0;
   L->y = round_up(phase, 256);
-  L->a = L->y + round_up((size_t)m * ymax * 4, 256);
+  // batch 1 (persistent kernel): one output region per phase type, the down
+  // phase's first so that L->y always holds the last phase's outputs
+  const size_t yb = round_up((size_t)m * ymax * 4, 256);
+  L->a = L->y + (m == 1 ? 4 : 1) * yb;
   L->b = L->a + round_up((size_t)m * amax * 2, 256);
   L->c = L->b + round_up((size_t)m * bmax * 2, 256);
   L->h = L->c + round_up((size_t)m * cmax * 2, 256);
   L->signs = L->h + round_up((size_t)m * hmax * 2, 256);
   L->sign_words = (uint32_t)words;
-  L->sync = L->signs + round_up((size_t)words * 4, 256);
+  L->params = L->signs + round_up((size_t)words * 4, 256);
+  L->straddle = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
+  L->sync = L->straddle + round_up((size_t)n_layers * 4 * kStackMaxCtas * sizeof(int2), 256);
   L->total = L->sync + 256;
   return TQ_OK;
 }
@@ -693,7 +701,7 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
 // too wide for shared memory.
 static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in, uint64_t seed,
                       uint16_t* h_out, char* ws, const StackWs& L, int sms, cudaStream_t s) {
-  if (n_layers > tq::STACK_MAX_LAYERS) return TQ_ERR_SHAPE;
+  if (n_layers > tq::STACK_MAX_LAYERS || sms > kStackMaxCtas) return TQ_ERR_SHAPE;
   static thread_local tq::StackParams sp;  // large (~25 KB): per-thread storage, copied into the launch
   memset(&sp, 0, sizeof(sp));
   const uint16_t* cb = layers[0].q.codebook_d;
@@ -721,7 +729,10 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
     }
   }
   const int lv = dmma_lv_for(true, kmax);
-  const size_t smem = (16384u << lv) + (size_t)kmax * 4 + sizeof(tq::DmmaParams) + 16;
+  const size_t smem = (16384u << lv) + (size_t)kmax * 4 + 4 * tq::PARAM_QUADS * 16 +
+                      tq::DMMA_WARPS * 32 * sizeof(float) + (size_t)sms * 16 * sizeof(uint16_t) +
+                      (size_t)kmax / 16 * sizeof(int32_t) + 2 * (size_t)sms * 2 * sizeof(int32_t) +
+                      4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) + 32;
   if (smem > 227 * 1024) return TQ_ERR_SHAPE;
   sp.n_layers = n_layers;
   sp.lv = lv;
@@ -732,7 +743,11 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.buf[1] = reinterpret_cast<uint16_t*>(ws + L.b);
   sp.buf[2] = reinterpret_cast<uint16_t*>(ws + L.c);
   sp.buf[3] = reinterpret_cast<uint16_t*>(ws + L.h);
-  sp.y = reinterpret_cast<float*>(ws + L.y);
+  {
+    const size_t yb = (L.a - L.y) / 4;  // one region per phase type: down, qkv, o, gate|up
+    const int order[4] = {1, 2, 3, 0};
+    for (int ph = 0; ph < 4; ++ph) sp.y[ph] = reinterpret_cast<float*>(ws + L.y + order[ph] * yb);
+  }
   sp.signs = reinterpret_cast<uint32_t*>(ws + L.signs);
   sp.sign_words = L.sign_words;
   sp.seed = seed;
@@ -740,6 +755,8 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.status = reinterpret_cast<int32_t*>(ws + kStatusOff);
   sp.partials = reinterpret_cast<float*>(ws + kCounterBytes);
   sp.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
+  sp.phase_table = reinterpret_cast<uint4*>(ws + L.params);
+  sp.straddle_table = reinterpret_cast<int2*>(ws + L.straddle);
   sp.spin_limit = 1u << 24;  // x 64 ns sleeps: ~1 s, far above any healthy phase
   void (*kern)(tq::StackParams);
   switch (lv) {
@@ -752,8 +769,8 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   int occ = 0;
   TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
   if (occ < 1) return TQ_ERR_SHAPE;
-  // partial sums: every warp of the grid may hold two tile partials
-  if ((size_t)sms * tq::DMMA_WARPS * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
+  // partial sums of straddling tiles: three phases x every CTA x two tiles
+  if ((size_t)3 * sms * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
   TQ_CUDA(cudaMemsetAsync(ws + L.sync, 0, 256, s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);

@@ -66,6 +66,8 @@ struct DmmaParams {
   int32_t blocks;          // k / 256
   int64_t units;           // tiles * blocks
   int32_t active_warps;
+  uint64_t rcp_active;     // floor((2^64 - 1) / active_warps), floor((2^64 - 1) / units):
+  uint64_t rcp_units;      // exact divisions by multiply-high (persistent stack kernel)
 };
 
 __host__ __device__ __forceinline__ int64_t dmma_warp_begin(int64_t w, int64_t units, int64_t active) {
@@ -198,18 +200,13 @@ __device__ __forceinline__ int partial_index(int g, int q, int jt, int i) {
   return row * MC + jt * 8 + 2 * q + (i & 1);
 }
 
+// A tile whose units span several warps: each contributor writes its partial
+// sum (slot 0 = the contributor's first tile, slot 1 = a later one), bumps the
+// tile's counter, and the last to arrive sums all of them in warp order.
 template <int NT, bool HILO>
-__device__ __forceinline__ void dmma_flush(const DmmaParams& p, int64_t W, int64_t wb, int64_t we, int t, int g,
-                                           int q, float (&acc)[NT][4]) {
+__device__ __forceinline__ void dmma_write_partial(const DmmaParams& p, int64_t W, int slot, int g, int q,
+                                                   const float (&acc)[NT][4]) {
   constexpr int MC = HILO ? 1 : NT * 8;
-  const int64_t B = p.blocks;
-  const int64_t t0 = (int64_t)t * B, t1 = t0 + B;
-  if (t0 >= wb && t1 <= we) {  // the whole tile ran in this warp
-    dmma_epilogue<NT, HILO>(p, t, g, q, acc);
-    return;
-  }
-  const int lane = threadIdx.x & 31;
-  const int slot = (t == (int)(wb / B)) ? 0 : 1;
   float* part = p.partials + ((size_t)W * 2 + slot) * (16 * MC);
   if (HILO) {
     if (q == 0) {
@@ -222,24 +219,32 @@ __device__ __forceinline__ void dmma_flush(const DmmaParams& p, int64_t W, int64
 #pragma unroll
       for (int i = 0; i < 4; ++i) part[partial_index<NT, HILO>(g, q, jt, i)] = acc[jt][i];
   }
-  __threadfence();
-  __syncwarp();
-  int old = 0;
-  if (lane == 0) old = atomicAdd(p.counters + t, 1);
-  old = __shfl_sync(0xffffffffu, old, 0);
+}
+
+// Called by the tile's last contributor (after its counter increment saw
+// every other one): sum the partials in warp order (grouped by CTA), write
+// y / handoff, and leave the counter at zero for the next call.
+template <int NT, bool HILO>
+__device__ __forceinline__ void dmma_reduce_tile(const DmmaParams& p, int t, int g, int q) {
+  constexpr int MC = HILO ? 1 : NT * 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t B = p.blocks;
+  const int64_t t0 = (int64_t)t * B, t1 = t0 + B;
   const int64_t wa = dmma_warp_of(t0, p.units, p.active_warps);
   const int64_t wz = dmma_warp_of(t1 - 1, p.units, p.active_warps);
-  if (old != (int)(wz - wa)) return;  // not the last contributor
   __threadfence();
-  // Sum the contributors in warp order.  Only the first contributor can have
-  // started before the tile (then the tile is its tail slot); every later one
-  // starts inside it (head slot).  Loads are issued CB contributors at a time.
+  // Only the first contributor can have started before the tile (then the
+  // tile is its slot 1); every later one starts inside it (slot 0).  Loads
+  // are issued CB contributors at a time.
   constexpr int CB = NT >= 8 ? 1 : 8 / NT;
-  float sum[NT][4];
+  // Partials are summed per group of DMMA_WARPS consecutive warps (one CTA)
+  // first, then the group sums in order: the same association as a two-level
+  // (CTA, then grid) reduction, so both give identical bits.
+  float sum[NT][4], gsum[NT][4];
 #pragma unroll
   for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sum[jt][i] = 0.f;
+    for (int i = 0; i < 4; ++i) sum[jt][i] = gsum[jt][i] = 0.f;
   const int first_slot = (dmma_warp_begin(wa, p.units, p.active_warps) >= t0) ? 0 : 1;
   const int ncontrib = (int)(wz - wa) + 1;
   for (int c0 = 0; c0 < ncontrib; c0 += CB) {
@@ -263,14 +268,59 @@ __device__ __forceinline__ void dmma_flush(const DmmaParams& p, int64_t W, int64
     }
 #pragma unroll
     for (int c = 0; c < CB; ++c)
-      if (c0 + c < ncontrib)
+      if (c0 + c < ncontrib) {
+        if (c0 + c > 0 && ((wa + c0 + c) % DMMA_WARPS) == 0) {  // next CTA-sized group
+#pragma unroll
+          for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              sum[jt][i] += gsum[jt][i];
+              gsum[jt][i] = 0.f;
+            }
+        }
 #pragma unroll
         for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sum[jt][i] += v[c][jt][i];
+          for (int i = 0; i < 4; ++i) gsum[jt][i] += v[c][jt][i];
+      }
   }
+#pragma unroll
+  for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sum[jt][i] += gsum[jt][i];
   dmma_epilogue<NT, HILO>(p, t, g, q, sum);
   if (lane == 0) p.counters[t] = 0;  // leave the counter ready for the next call
+}
+
+// Number of warps whose unit ranges meet tile t.
+__device__ __forceinline__ int dmma_contributors(const DmmaParams& p, int t) {
+  const int64_t t0 = (int64_t)t * p.blocks, t1 = t0 + p.blocks;
+  return (int)(dmma_warp_of(t1 - 1, p.units, p.active_warps) - dmma_warp_of(t0, p.units, p.active_warps)) + 1;
+}
+
+// End of a warp's unit range: publish the (at most two) tiles it shares with
+// other warps -- the first tile of the range (its sums kept in registers
+// since that tile ended) and the last -- with ONE fence, then finish the ones
+// this warp was last to reach.  Deferring the first tile keeps the fence and
+// the counter round trip out of the code stream.
+template <int NT, bool HILO>
+__device__ __forceinline__ void dmma_publish(const DmmaParams& p, int64_t W, int g, int q, bool has_head, int head_t,
+                                             const float (&hacc)[NT][4], bool has_tail, int tail_t, int tail_slot,
+                                             const float (&tacc)[NT][4]) {
+  const int lane = threadIdx.x & 31;
+  if (has_head) dmma_write_partial<NT, HILO>(p, W, 0, g, q, hacc);
+  if (has_tail) dmma_write_partial<NT, HILO>(p, W, tail_slot, g, q, tacc);
+  __threadfence();
+  __syncwarp();
+  int oh = 0, ot = 0;
+  if (lane == 0) {
+    if (has_head) oh = atomicAdd(p.counters + head_t, 1);
+    if (has_tail) ot = atomicAdd(p.counters + tail_t, 1);
+  }
+  oh = __shfl_sync(0xffffffffu, oh, 0);
+  ot = __shfl_sync(0xffffffffu, ot, 0);
+  if (has_head && oh == dmma_contributors(p, head_t) - 1) dmma_reduce_tile<NT, HILO>(p, head_t, g, q);
+  if (has_tail && ot == dmma_contributors(p, tail_t) - 1) dmma_reduce_tile<NT, HILO>(p, tail_t, g, q);
 }
 
 // Replicate the codebook into V = 2^LV shared-memory views (entry e of view
@@ -329,9 +379,13 @@ __device__ __forceinline__ uint2 lds_b_hilo(const uint8_t* addr, int lane) {
 
 // The unit loop of one warp: decode its units, run the MMAs, flush tiles.
 // `smem` holds the codebook views, `xs` the batch-1 activations (hi/lo).
+// With `wslots` (batch 1 only) the tiles this warp shares with other warps
+// are not published through global memory: their partial sums go to this
+// warp's two shared-memory slots ([2][16] floats, slot 0 = the range's first
+// tile), for a reduction by the whole CTA.
 template <int LV, int NT, bool HILO>
 __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* smem, const uint8_t* xs, int64_t W,
-                                           DmmaCursor& c, int lane) {
+                                           DmmaCursor& c, int lane, float* wslots = nullptr) {
   constexpr int V = 1 << LV;
   constexpr int SH = 3 + LV;
   const int g = lane >> 2, q = lane & 3;
@@ -348,6 +402,13 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
     for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
 
   const int nunits = (int)(c.we - c.wb);
+  bool has_head = false, has_tail = false;
+  int head_t = 0, tail_t = 0;
+  float hacc[NT][4];
+#pragma unroll
+  for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hacc[jt][i] = 0.f;
   for (int iu = 0; iu < nunits; ++iu) {
     int tn = t, bn = b + 1;
     if (bn == p.blocks) {
@@ -407,21 +468,60 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
       }
     }
 
-    if (iu + 1 == nunits || bn == 0) {
+    if (iu + 1 == nunits || bn == 0) {  // tile t ends here (for this warp)
 #pragma unroll
       for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[jt][i] += acc2[jt][i];
-      dmma_flush<NT, HILO>(p, W, c.wb, c.we, t, g, q, acc);
+      const int64_t t0 = (int64_t)t * p.blocks;
+      if (t0 >= c.wb && t0 + p.blocks <= c.we) {
+        dmma_epilogue<NT, HILO>(p, t, g, q, acc);  // the whole tile ran in this warp
+      } else if (iu + 1 < nunits) {
+        // the range's first tile, shared with earlier warps: publish it at the
+        // end (8 column tiles keep no second register copy: publish now)
+        if (NT <= 4) {
+          has_head = true;
+          head_t = t;
 #pragma unroll
-      for (int jt = 0; jt < NT; ++jt)
+          for (int jt = 0; jt < NT; ++jt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
+            for (int i = 0; i < 4; ++i) hacc[jt][i] = acc[jt][i];
+        } else {
+          dmma_publish<NT, HILO>(p, W, g, q, true, t, acc, false, 0, 0, acc);
+        }
+      } else {
+        has_tail = true;
+        tail_t = t;
+      }
+      if (iu + 1 < nunits || !has_tail) {
+#pragma unroll
+        for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
+      }
     }
     t = tn;
     b = bn;
     rows = nrows;
     cur = nxt;
+  }
+  if (has_head || has_tail) {
+    // slot 0 holds the range's first tile, slot 1 a later one
+    const int tail_slot = (tail_t == (int)(c.wb / p.blocks)) ? 0 : 1;
+    if (HILO && wslots) {
+      if (q == 0) {
+        if (has_head) {
+          wslots[g] = hacc[0][0] + hacc[0][1];
+          wslots[g + 8] = hacc[0][2] + hacc[0][3];
+        }
+        if (has_tail) {
+          wslots[tail_slot * 16 + g] = acc[0][0] + acc[0][1];
+          wslots[tail_slot * 16 + g + 8] = acc[0][2] + acc[0][3];
+        }
+      }
+    } else {
+      dmma_publish<NT, HILO>(p, W, g, q, has_head, head_t, hacc, has_tail, tail_t, tail_slot, acc);
+    }
   }
 }
 

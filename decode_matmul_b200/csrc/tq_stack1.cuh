@@ -6,13 +6,18 @@
 // ("8 open models" article, "Speed": batch-1 generation is one read of the
 // weights per token).  Here one cooperative launch (one CTA per SM) runs
 // every phase of every layer:
-//   * the codebook views are built once; the RHT sign bits of every phase
-//     are drawn once into a table;
+//   * the codebook views are built once; the RHT sign bits and the unit
+//     split of every phase are computed once into tables;
 //   * between phases a grid barrier (atomic arrive + bounded acquire poll)
-//     orders the handoff of phase f before the RHT of phase f+1; each warp
+//     orders the outputs of phase f before the RHT of phase f+1; each warp
 //     loads the first code chunk of phase f+1 before waiting at the barrier;
-//   * each phase is the same warp-level unit split and deterministic
-//     last-arriver reduction as the single-phase kernel.
+//   * units are split over warps exactly as in the single-phase kernel, but
+//     the reduction has two levels and no global round trip inside a phase:
+//     warps that share a tile leave their partial sums in shared memory and
+//     the CTA sums them; a tile that straddles CTAs leaves one partial per
+//     CTA in global memory, and the next phase sums those (in CTA order)
+//     while it loads its input, after the barrier.  Grouping the sums by CTA
+//     gives the same bits as the single-phase kernel's last-arriver sum.
 // Every wait is bounded: on timeout the kernel records TQ_ERR_TIMEOUT in the
 // status word and all CTAs leave.
 #pragma once
@@ -23,6 +28,8 @@ namespace tq {
 
 constexpr int STACK_MAX_LAYERS = 128;
 constexpr int STACK_TIMEOUT_STATUS = 7;  // TQ_ERR_TIMEOUT
+
+constexpr int PARAM_QUADS = (int)((sizeof(DmmaParams) + 15) / 16);  // 16-byte words of one DmmaParams
 
 struct StackLayerDev {
   const uint8_t* codes[7];  // q k v o gate up down
@@ -41,13 +48,15 @@ struct StackParams {
   const uint16_t* h_in;
   uint16_t* h_out;
   uint16_t* buf[4];       // phase handoffs: q, o, gate, layer output
-  float* y;               // every phase's outputs (k, v and up land here)
+  float* y[4];            // outputs of each phase type (k, v and up land here too)
   uint32_t* signs;        // sign bits, bit set = the diagonal entry is -1
   uint32_t sign_words;
   uint64_t seed;
-  float* partials;
+  float* partials;        // per-CTA partials of straddling tiles: [3][grid][2][16]
   int32_t* counters;
   uint32_t* sync;         // barrier counter, zero at launch
+  uint4* phase_table;     // [4 * n_layers][PARAM_QUADS]: every phase's parameters
+  int2* straddle_table;   // [4 * n_layers][grid]: every phase's straddling-tile entries
   int32_t* status;
   uint32_t spin_limit;
 };
@@ -56,29 +65,6 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
   return v;
-}
-
-// RHT of one 512-block with the diagonal taken from the sign table.  The
-// input and the table were written by other CTAs of this launch, so they are
-// read through L2 (ld.global.cg), never from a possibly stale L1 line.
-__device__ __forceinline__ void rht512_warp_table(const uint16_t* x, int blk, const uint32_t* signs, float v[16]) {
-  const int lane = threadIdx.x & 31;
-  const int base = blk * 512 + lane * 16;
-  const uint4* src = reinterpret_cast<const uint4*>(x + base);
-  const uint4 p0 = __ldcg(src), p1 = __ldcg(src + 1);
-  const uint32_t bits = __ldcg(signs + (base >> 5)) >> (base & 16);
-  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = (w[i] & 0xFFFFu) ^ (((bits >> (2 * i)) & 1u) << 15);
-    const uint32_t hi = (w[i] >> 16) ^ (((bits >> (2 * i + 1)) & 1u) << 15);
-    v[2 * i] = bf16_bits_to_f(lo);
-    v[2 * i + 1] = bf16_bits_to_f(hi);
-  }
-  wht512_warp(v);
-  const float inv = 0.044194173824159216f;  // 1/sqrt(512)
-#pragma unroll
-  for (int r = 0; r < 16; ++r) v[r] *= inv;
 }
 
 // Phase f = 4l + p as single-phase parameters.
@@ -105,7 +91,7 @@ __device__ __forceinline__ void stack_phase_params(const StackParams& sp, int f,
   p.x_f16 = nullptr;
   p.x_bf16 = ph == 0 ? (l == 0 ? sp.h_in : sp.buf[3]) : sp.buf[ph - 1];
   p.rht_seed = 0;
-  p.y = sp.y;
+  p.y = sp.y[ph];
   p.handoff = (ph == 3 && l == sp.n_layers - 1) ? sp.h_out : sp.buf[ph];
   p.handoff_rows = L.n[first];
   p.alpha = L.alpha[ph];
@@ -115,6 +101,8 @@ __device__ __forceinline__ void stack_phase_params(const StackParams& sp, int f,
   p.blocks = p.k / 256;
   p.units = (int64_t)p.tiles * p.blocks;
   p.active_warps = (int32_t)(p.units < grid_warps ? p.units : grid_warps);
+  p.rcp_active = ~0ULL / (uint64_t)p.active_warps;
+  p.rcp_units = ~0ULL / (uint64_t)p.units;
 }
 
 // Arrive at the grid barrier (after the whole CTA finished its writes).
@@ -143,6 +131,258 @@ __device__ __forceinline__ bool grid_wait(const StackParams& sp, uint32_t target
   return *abort_flag == 0;
 }
 
+// floor(n / d) for n < 2^53 and 0 < d < 2^32, given r = floor((2^64 - 1) / d):
+// the multiply-high is floor(n / d) or one less (the error of r is below
+// n / 2^64 < 1), and one step corrects it.
+__device__ __forceinline__ uint64_t div_rcp(uint64_t n, uint64_t d, uint64_t r) {
+  uint64_t q = __umul64hi(n, r);
+  if ((q + 1) * d <= n) ++q;
+  return q;
+}
+
+// The unit split of dmma_warp_begin / dmma_warp_of, per warp and per CTA
+// (CTA c holds warps DMMA_WARPS*c .. DMMA_WARPS*c + DMMA_WARPS-1).
+__device__ __forceinline__ int64_t sk_warp_begin(const DmmaParams& p, int64_t w) {
+  return (int64_t)div_rcp((uint64_t)w * (uint64_t)p.units, (uint64_t)p.active_warps, p.rcp_active);
+}
+__device__ __forceinline__ int64_t sk_cta_begin(const DmmaParams& p, int c) {
+  return sk_warp_begin(p, min((int64_t)c * DMMA_WARPS, (int64_t)p.active_warps));
+}
+__device__ __forceinline__ int sk_cta_of(const DmmaParams& p, int64_t u) {
+  const uint64_t w = div_rcp((uint64_t)(u + 1) * (uint64_t)p.active_warps + (uint64_t)p.units - 1,
+                             (uint64_t)p.units, p.rcp_units) - 1;
+  return (int)(w / DMMA_WARPS);
+}
+
+// y and handoff of one output row.
+__device__ __forceinline__ void stack_store_row(const DmmaParams& p, int R, float v) {
+  if (R < p.n_total) {
+    if (p.y) p.y[R] = v;
+    if (R < p.handoff_rows) p.handoff[R] = f_to_bf16_bits(p.alpha * v);
+  }
+}
+
+// After the unit loop and a __syncthreads: the tiles this CTA touched that no
+// single warp finished.  Warp w's partial of tile t sits in its slot 0 when t
+// is the first tile of its range, else in slot 1.  A tile inside the CTA is
+// summed here in warp order and written; a tile that straddles CTAs leaves
+// the CTA's sum in gp[cta][s] (s = 0 for the CTA's first tile, 1 for its
+// last) for the next phase.  `wbeg` = first unit of each warp of the CTA
+// (17 entries), `wfirst` = first tile of each warp.
+__device__ __forceinline__ void stack_cta_reduce(const DmmaParams& p, const int32_t* wbeg, const int32_t* wfirst,
+                                                 const float* wslots, float* gp, int warp, int lane) {
+  const int32_t b0 = wbeg[0], b1 = wbeg[DMMA_WARPS];
+  if (b0 >= b1) return;
+  const int32_t B = p.blocks;
+  const int T0 = wfirst[0], T1 = (b1 - 1) / B;
+  const int lw = lane & (DMMA_WARPS - 1);
+  const int32_t lb = wbeg[lw], le = wbeg[lw + 1], lf = wfirst[lw];
+  for (int t = T0 + warp; t <= T1; t += DMMA_WARPS) {
+    const int32_t t0 = t * B, t1 = t0 + B;
+    // warps of this CTA whose (non-empty) ranges meet the tile
+    const uint32_t meet = __ballot_sync(0xffffffffu, lane < DMMA_WARPS && lb < le && lb < t1 && le > t0);
+    const int wa = __ffs(meet) - 1, wz = 31 - __clz(meet);
+    const bool one = wa == wz && __shfl_sync(0xffffffffu, lb, wa) <= t0 && __shfl_sync(0xffffffffu, le, wa) >= t1;
+    if (one) continue;  // finished by that warp
+    // this lane's contributor slot: every contributor's value is loaded, then summed in warp order
+    const int ls = (lf == t) ? 0 : 1;
+    float v = 0.f;
+    if (lane < 16) {
+      float part[DMMA_WARPS];
+#pragma unroll
+      for (int w = 0; w < DMMA_WARPS; ++w) {
+        const int sw = __shfl_sync(0x0000ffffu, ls, w);
+        part[w] = (w >= wa && w <= wz) ? wslots[(w * 2 + sw) * 16 + lane] : 0.f;
+      }
+#pragma unroll
+      for (int w = 0; w < DMMA_WARPS; ++w)
+        if (w >= wa && w <= wz) v += part[w];
+      if (t0 >= b0 && t1 <= b1) {
+        // the association of the single-phase kernel: (0 + group sum) + 0
+        stack_store_row(p, t * 16 + lane, (0.f + v) + 0.f);
+      } else {
+        __stcg(gp + ((size_t)blockIdx.x * 2 + (t == T0 ? 0 : 1)) * 16 + lane, v);
+      }
+    }
+  }
+}
+
+// The previous phase's tiles (parameters q, CTA partials gq) that straddle
+// CTAs.  Tile T is taken once, under the CTA c where it starts (T is then the
+// last tile of c's range): sent[c] = {T, cz | s0 << 16} (T < 0: none), with
+// cz the last contributing CTA and s0 the slot of c's partial.  Its value is
+// the sum over the contributing CTAs c .. cz in order.  Rows of the consumed
+// op (the handoff) go, rounded as the handoff is, to fixb[c][16] with
+// tmap[T] = f << 16 | c, for the RHT of this phase; CTA c alone writes the
+// outputs (y, handoff) of entry c.  With fixb == nullptr only those writes
+// are done.
+__device__ __forceinline__ void stack_fixups(const DmmaParams& q, const int2* sent, const float* gq, uint16_t* fixb,
+                                             int32_t* tmap, int f, int tid) {
+  const int grid = gridDim.x;
+  for (int task = tid; task < grid * 2; task += DMMA_THREADS) {  // one pass for grids up to 256 CTAs
+    const int c = task >> 1, h = task & 1;                         // rows 8h .. 8h+7 of the tile
+    const bool writer = c == (int)blockIdx.x;
+    if (!fixb && !writer) continue;
+    const int2 e = sent[c];
+    if (e.x < 0) continue;
+    const int T = e.x, cz = e.y & 0xFFFF, s0 = e.y >> 16;
+    const bool consumed = fixb && T * 16 < q.handoff_rows;
+    if (!consumed && !writer) continue;
+    float4 v[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4* src = reinterpret_cast<const float4*>(gq + ((size_t)(c + i) * 2 + (i ? 0 : s0)) * 16) + 2 * h;
+      const bool live = c + i <= cz;
+      v[i][0] = live ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[i][1] = live ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float acc[8];
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) acc[e8] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (c + i <= cz) {
+        const float* vv = reinterpret_cast<const float*>(&v[i][0]);
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) acc[e8] += vv[e8];
+      }
+    for (int cc = c + 4; cc <= cz; ++cc) {  // a tile over more than four CTAs
+      const float4* src = reinterpret_cast<const float4*>(gq + (size_t)cc * 2 * 16) + 2 * h;
+      const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
+      acc[0] += u0.x;
+      acc[1] += u0.y;
+      acc[2] += u0.z;
+      acc[3] += u0.w;
+      acc[4] += u1.x;
+      acc[5] += u1.y;
+      acc[6] += u1.z;
+      acc[7] += u1.w;
+    }
+#pragma unroll
+    for (int e8 = 0; e8 < 8; ++e8) {
+      const float fin = acc[e8] + 0.f;
+      if (consumed) fixb[c * 16 + h * 8 + e8] = f_to_bf16_bits(q.alpha * fin);
+      if (writer) stack_store_row(q, T * 16 + h * 8 + e8, fin);
+    }
+    if (consumed && h == 0) tmap[T] = (f << 16) | c;
+  }
+}
+
+// RHT of one 512-block with the diagonal taken from the sign table, in two
+// steps so that a warp issues the loads of all its blocks before the first
+// transform.  The input and the table were written by other CTAs of this
+// launch, so they are read through L2 (ld.global.cg), never from a possibly
+// stale L1 line.
+struct RhtIn {
+  uint4 p0, p1;
+  uint32_t bits;
+};
+
+__device__ __forceinline__ RhtIn rht_table_load(const uint16_t* x, int blk, const uint32_t* signs) {
+  const int lane = threadIdx.x & 31;
+  const int base = blk * 512 + lane * 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x + base);
+  RhtIn r;
+  r.p0 = __ldcg(src);
+  r.p1 = __ldcg(src + 1);
+  r.bits = __ldcg(signs + (base >> 5)) >> (base & 16);
+  return r;
+}
+
+// Transform block blk and store it as hi/lo quads.  When tmap marks this
+// lane's 16 inputs (one tile of the previous phase) as summed in this phase,
+// they come from fixb instead of the handoff in global memory.
+__device__ __forceinline__ void rht_table_finish(RhtIn r, int blk, const uint16_t* fixb, const int32_t* tmap, int f,
+                                                 uint8_t* xs) {
+  const int lane = threadIdx.x & 31;
+  if (tmap) {
+    const int32_t tg = tmap[blk * 32 + lane];
+    if ((tg >> 16) == f) {
+      const uint4* src = reinterpret_cast<const uint4*>(fixb + (tg & 0xFFFF) * 16);
+      r.p0 = src[0];
+      r.p1 = src[1];
+    }
+  }
+  const uint32_t w[8] = {r.p0.x, r.p0.y, r.p0.z, r.p0.w, r.p1.x, r.p1.y, r.p1.z, r.p1.w};
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = bf16_bits_to_f((w[i] & 0xFFFFu) ^ (((r.bits >> (2 * i)) & 1u) << 15));
+    v[2 * i + 1] = bf16_bits_to_f((w[i] >> 16) ^ (((r.bits >> (2 * i + 1)) & 1u) << 15));
+  }
+  wht512_warp(v);
+  const float inv = 0.044194173824159216f;  // 1/sqrt(512)
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] *= inv;
+#pragma unroll
+  for (int r4 = 0; r4 < 4; ++r4)
+    store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
+}
+
+// The phase's activations x' = RHT(x) as hi/lo fp16 quads in shared memory.
+// Block blk goes to warp blk % 16 and up to three blocks per warp have their
+// loads in flight together; meanwhile the CTA sums the previous phase's
+// straddling tiles (q != nullptr, entries sentq) and then fills the next
+// phase's warp tables (pn != nullptr).  Ends with a __syncthreads.
+__device__ __forceinline__ void stack_warp_tables(const DmmaParams& p, int32_t* wbeg, int32_t* wfirst, int tid);
+
+__device__ __forceinline__ void stack_rht(const DmmaParams& p, const DmmaParams* q, const int2* sentq, const float* gq,
+                                          const uint32_t* signs, uint8_t* xs, uint16_t* fixb, int32_t* tmap, int f,
+                                          int tid, const DmmaParams* pn, int32_t* wbegn, int32_t* wfirstn) {
+  const int warp = tid >> 5;
+  const int nb = p.k / 512;
+  RhtIn in[3];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+    if (warp + DMMA_WARPS * r < nb) in[r] = rht_table_load(p.x_bf16, warp + DMMA_WARPS * r, signs);
+  if (q) stack_fixups(*q, sentq, gq, fixb, tmap, f, tid);
+  __syncthreads();
+  if (pn) stack_warp_tables(*pn, wbegn, wfirstn, tid);  // the next phase's
+  const int32_t* tm = q ? tmap : nullptr;
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+    if (warp + DMMA_WARPS * r < nb) rht_table_finish(in[r], warp + DMMA_WARPS * r, fixb, tm, f, xs);
+  for (int blk = warp + 3 * DMMA_WARPS; blk < nb; blk += DMMA_WARPS)  // k > 24576 only
+    rht_table_finish(rht_table_load(p.x_bf16, blk, signs), blk, fixb, tm, f, xs);
+  __syncthreads();
+}
+
+// The straddling tile entered under CTA c in phase p (see stack_fixups).
+__device__ __forceinline__ int2 stack_straddle_entry(const DmmaParams& p, int c) {
+  const int64_t B = p.blocks;
+  const int64_t b0 = sk_cta_begin(p, c), b1 = sk_cta_begin(p, c + 1);
+  int2 e = make_int2(-1, 0);
+  if (b0 < b1) {
+    const int64_t T = (b1 - 1) / B, t0 = T * B, t1 = t0 + B;
+    if (t0 >= b0 && t1 > b1) e = make_int2((int)T, sk_cta_of(p, t1 - 1) | ((b0 / B == T) ? 0 : 1) << 16);
+  }
+  return e;
+}
+
+// First unit and first tile of each warp of this CTA in phase p.
+__device__ __forceinline__ void stack_warp_tables(const DmmaParams& p, int32_t* wbeg, int32_t* wfirst, int tid) {
+  if (tid <= DMMA_WARPS) {
+    const int64_t w = min((int64_t)blockIdx.x * DMMA_WARPS + tid, (int64_t)p.active_warps);
+    const int32_t b = (int32_t)sk_warp_begin(p, w);
+    wbeg[tid] = b;
+    wfirst[tid] = b / p.blocks;
+  }
+}
+
+// dmma_begin with the unit range of this warp taken from the tables.
+__device__ __forceinline__ void stack_begin(const DmmaParams& p, const int32_t* wbeg, const int32_t* wfirst, int warp,
+                                            int lane, DmmaCursor& c) {
+  c.wb = wbeg[warp];
+  c.we = wbeg[warp + 1];
+  c.t = c.b = 0;
+  if (c.wb < c.we) {
+    c.t = wfirst[warp];
+    c.b = (int)(c.wb - (int64_t)c.t * p.blocks);
+    c.rows = dmma_rows(p, c.t, lane >> 2, lane & 3);
+    c.cur = dmma_fetch(c.rows, c.b);
+  }
+}
+
 template <int LV>
 __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_constant__ StackParams sp) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -150,14 +390,50 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
   int kmax = 0;
   for (int l = 0; l < sp.n_layers; ++l)
     for (int ph = 0; ph < 4; ++ph) kmax = max(kmax, sp.layers[l].k[ph]);
-  DmmaParams* pp = reinterpret_cast<DmmaParams*>(xs + (size_t)kmax * 4);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(pp + 1);
+  // four parameter slots: previous, running, next and next-but-one phase
+  uint4* slots = reinterpret_cast<uint4*>(xs + (size_t)kmax * 4);
+  float* wslots = reinterpret_cast<float*>(slots + 4 * PARAM_QUADS);      // [warp][2][16]
+  uint16_t* fixb = reinterpret_cast<uint16_t*>(wslots + DMMA_WARPS * 32);  // [grid][16]
+  int32_t* tmap = reinterpret_cast<int32_t*>(fixb + gridDim.x * 16);       // [kmax / 16]
+  int2* sentt = reinterpret_cast<int2*>(tmap + kmax / 16);                 // [2][grid]
+  int32_t* wbegt = reinterpret_cast<int32_t*>(sentt + 2 * gridDim.x);      // [2][DMMA_WARPS + 1]
+  int32_t* wfirstt = wbegt + 2 * (DMMA_WARPS + 1);                         // [2][DMMA_WARPS + 1]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(wfirstt + 2 * (DMMA_WARPS + 1));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int grid_warps = gridDim.x * DMMA_WARPS;
   const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
   const int nphases = 4 * sp.n_layers;
+  const size_t gstride = (size_t)gridDim.x * 32;  // floats of one phase's CTA partials
+  auto slot = [&](int f) -> DmmaParams& { return *reinterpret_cast<DmmaParams*>(slots + (f & 3) * PARAM_QUADS); };
+  auto sentf = [&](int f) { return sentt + (f & 1) * gridDim.x; };
+  auto wbeg = [&](int f) { return wbegt + (f & 1) * (DMMA_WARPS + 1); };
+  auto wfirst = [&](int f) { return wfirstt + (f & 1) * (DMMA_WARPS + 1); };
 
-  if (tid == 0) *abort_flag = 0;
+  if (tid == 0) {
+    *abort_flag = 0;
+    stack_phase_params(sp, 0, slot(0), grid_warps);
+  }
+  if (tid == 32 && nphases > 1) stack_phase_params(sp, 1, slot(1), grid_warps);
+  for (int i = tid; i < kmax / 16; i += DMMA_THREADS) tmap[i] = -1;
+  // every phase's parameters, one thread each, into the table read later
+  for (int f = blockIdx.x * DMMA_THREADS + tid; f < nphases; f += gridDim.x * DMMA_THREADS) {
+    DmmaParams pf;
+    stack_phase_params(sp, f, pf, grid_warps);
+    const uint4* src = reinterpret_cast<const uint4*>(&pf);
+    for (int i = 0; i < (int)(sizeof(DmmaParams) / 16); ++i) sp.phase_table[(size_t)f * PARAM_QUADS + i] = src[i];
+    if (sizeof(DmmaParams) % 16) {
+      uint4 tail = make_uint4(0u, 0u, 0u, 0u);
+      memcpy(&tail, reinterpret_cast<const uint8_t*>(&pf) + (sizeof(DmmaParams) / 16) * 16, sizeof(DmmaParams) % 16);
+      sp.phase_table[(size_t)f * PARAM_QUADS + sizeof(DmmaParams) / 16] = tail;
+    }
+  }
+  // every phase's straddling-tile entries, one (phase, CTA) per thread
+  for (int i = blockIdx.x * DMMA_THREADS + tid; i < nphases * (int)gridDim.x; i += gridDim.x * DMMA_THREADS) {
+    const int f = i / gridDim.x;
+    DmmaParams pf;
+    stack_phase_params(sp, f, pf, grid_warps);
+    sp.straddle_table[i] = stack_straddle_entry(pf, i - f * gridDim.x);
+  }
   build_views<LV>(smem, sp.codebook, tid, DMMA_THREADS);
 
   // RHT sign table: word j holds d[32j .. 32j+31] of the phase it belongs to.
@@ -173,38 +449,47 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     for (int i = 0; i < 32; ++i) bits |= (rht_sign_negative(seed_lp, k0 + i) ? 1u : 0u) << i;
     sp.signs[j] = bits;
   }
-  grid_arrive(sp);
+  grid_arrive(sp);  // its __syncthreads publishes slot 0 to the CTA
   uint32_t epoch = 1;
 
-  // first phase's parameters and code chunk, then the barrier
-  if (tid == 0) stack_phase_params(sp, 0, *pp, grid_warps);
+  // first phase's tables and code chunk, then the barrier
+  stack_warp_tables(slot(0), wbeg(0), wfirst(0), tid);
+  for (int c = tid; c < (int)gridDim.x; c += DMMA_THREADS) sentf(0)[c] = __ldcg(sp.straddle_table + c);
   __syncthreads();
   DmmaCursor c;
-  dmma_begin(*pp, W, lane >> 2, lane & 3, c);
+  stack_begin(slot(0), wbeg(0), wfirst(0), warp, lane, c);
   if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;
 
   for (int f = 0; f < nphases; ++f) {
     const int l = f >> 2, ph = f & 3;
-    // batch-1 activations of this phase: RHT with the table, hi/lo split
-    const uint32_t* sg = sp.signs + sp.layers[l].sign_off[ph];
-    for (int blk = warp; blk < pp->k / 512; blk += DMMA_WARPS) {
-      float v[16];
-      rht512_warp_table(pp->x_bf16, blk, sg, v);
-#pragma unroll
-      for (int r4 = 0; r4 < 4; ++r4)
-        store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
-    }
+    const DmmaParams& p = slot(f);
+    // parameters of phase f+2 come from the table while the RHT runs
+    uint4 nq = make_uint4(0u, 0u, 0u, 0u);
+    const bool fetch = tid < PARAM_QUADS && f + 2 < nphases;
+    if (fetch) nq = __ldcg(sp.phase_table + (size_t)(f + 2) * PARAM_QUADS + tid);
+    const bool next = f + 1 < nphases;
+    // and this phase's straddling entries (read by the next phase's RHT)
+    int2 se = make_int2(-1, 0);
+    if (f > 0 && tid < (int)gridDim.x) se = __ldcg(sp.straddle_table + (size_t)f * gridDim.x + tid);
+    stack_rht(p, f > 0 ? &slot(f - 1) : nullptr, sentf(f - 1), sp.partials + (size_t)((f + 2) % 3) * gstride,
+              sp.signs + sp.layers[l].sign_off[ph], xs, fixb, tmap, f, tid, next ? &slot(f + 1) : nullptr,
+              wbeg(f + 1), wfirst(f + 1));
+    if (fetch) slots[((f + 2) & 3) * PARAM_QUADS + tid] = nq;  // slot of phase f-2: no reader left
+    if (f > 0 && tid < (int)gridDim.x) sentf(f)[tid] = se;      // the previous phase's were read above
+    dmma_units<LV, 1, true>(p, smem, xs, W, c, lane, wslots + warp * 32);
     __syncthreads();
-    dmma_units<LV, 1, true>(*pp, smem, xs, W, c, lane);
-    grid_arrive(sp);
+    stack_cta_reduce(p, wbeg(f), wfirst(f), wslots, sp.partials + (size_t)(f % 3) * gstride, warp, lane);
+    grid_arrive(sp);  // its __syncthreads ends every use of the warp tables and slots
     ++epoch;
     if (f + 1 == nphases) break;
-    // next phase: parameters and first code chunk before the barrier wait
-    if (tid == 0) stack_phase_params(sp, f + 1, *pp, grid_warps);
-    __syncthreads();
-    dmma_begin(*pp, W, lane >> 2, lane & 3, c);
+    // next phase: first code chunk before the barrier wait
+    stack_begin(slot(f + 1), wbeg(f + 1), wfirst(f + 1), warp, lane, c);
     if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;
   }
+  // the last phase's straddling tiles: summed once every CTA partial is in
+  if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;
+  stack_fixups(slot(nphases - 1), sentf(nphases - 1),
+               sp.partials + (size_t)((nphases - 1) % 3) * gstride, nullptr, nullptr, nphases, tid);
 }
 
 }  // namespace tq
