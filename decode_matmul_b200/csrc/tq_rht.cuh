@@ -32,11 +32,12 @@ __device__ __forceinline__ void wht512_warp(float v[16]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
+    // upper lane: o - v, lower lane: v + o -- one exact fma with a +-1 factor
+    const float sg = (lane & m) ? -1.f : 1.f;
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
-      float o = __shfl_xor_sync(0xffffffffu, v[r], m);
-      v[r] = upper ? (o - v[r]) : (v[r] + o);
+      const float o = __shfl_xor_sync(0xffffffffu, v[r], m);
+      v[r] = fmaf(sg, v[r], o);
     }
   }
 }

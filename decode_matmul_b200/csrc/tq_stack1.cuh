@@ -454,7 +454,6 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
 
   // first phase's tables and code chunk, then the barrier
   stack_warp_tables(slot(0), wbeg(0), wfirst(0), tid);
-  for (int c = tid; c < (int)gridDim.x; c += DMMA_THREADS) sentf(0)[c] = __ldcg(sp.straddle_table + c);
   __syncthreads();
   DmmaCursor c;
   stack_begin(slot(0), wbeg(0), wfirst(0), warp, lane, c);
@@ -468,14 +467,15 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     const bool fetch = tid < PARAM_QUADS && f + 2 < nphases;
     if (fetch) nq = __ldcg(sp.phase_table + (size_t)(f + 2) * PARAM_QUADS + tid);
     const bool next = f + 1 < nphases;
-    // and this phase's straddling entries (read by the next phase's RHT)
+    // and this phase's straddling entries (read by the next phase's RHT;
+    // the table was written by all CTAs before the first barrier)
     int2 se = make_int2(-1, 0);
-    if (f > 0 && tid < (int)gridDim.x) se = __ldcg(sp.straddle_table + (size_t)f * gridDim.x + tid);
+    if (tid < (int)gridDim.x) se = __ldcg(sp.straddle_table + (size_t)f * gridDim.x + tid);
     stack_rht(p, f > 0 ? &slot(f - 1) : nullptr, sentf(f - 1), sp.partials + (size_t)((f + 2) % 3) * gstride,
               sp.signs + sp.layers[l].sign_off[ph], xs, fixb, tmap, f, tid, next ? &slot(f + 1) : nullptr,
               wbeg(f + 1), wfirst(f + 1));
     if (fetch) slots[((f + 2) & 3) * PARAM_QUADS + tid] = nq;  // slot of phase f-2: no reader left
-    if (f > 0 && tid < (int)gridDim.x) sentf(f)[tid] = se;      // the previous phase's were read above
+    if (tid < (int)gridDim.x) sentf(f)[tid] = se;      // the previous phase's were read above
     dmma_units<LV, 1, true>(p, smem, xs, W, c, lane, wslots + warp * 32);
     __syncthreads();
     stack_cta_reduce(p, wbeg(f), wfirst(f), wslots, sp.partials + (size_t)(f % 3) * gstride, warp, lane);
