@@ -769,8 +769,8 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   int occ = 0;
   TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
   if (occ < 1) return TQ_ERR_SHAPE;
-  // partial sums of straddling tiles: three phases x every CTA x two tiles
-  if ((size_t)3 * sms * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
+  // partial sums of straddling tiles: three phases x copies x every CTA x two tiles
+  if ((size_t)3 * tq::STACK_PART_COPIES * sms * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
   TQ_CUDA(cudaMemsetAsync(ws + L.sync, 0, 256, s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);

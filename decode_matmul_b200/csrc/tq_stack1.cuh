@@ -29,6 +29,11 @@ namespace tq {
 constexpr int STACK_MAX_LAYERS = 128;
 constexpr int STACK_TIMEOUT_STATUS = 7;  // TQ_ERR_TIMEOUT
 
+// Copies of each CTA partial of a straddling tile: every CTA reads all of
+// them after a barrier, and spreading the readers over copies keeps them off
+// the same L2 lines.
+constexpr int STACK_PART_COPIES = 8;
+
 constexpr int PARAM_QUADS = (int)((sizeof(DmmaParams) + 15) / 16);  // 16-byte words of one DmmaParams
 
 struct StackLayerDev {
@@ -52,7 +57,7 @@ struct StackParams {
   uint32_t* signs;        // sign bits, bit set = the diagonal entry is -1
   uint32_t sign_words;
   uint64_t seed;
-  float* partials;        // per-CTA partials of straddling tiles: [3][grid][2][16]
+  float* partials;        // per-CTA partials of straddling tiles: [3][STACK_PART_COPIES][grid][2][16]
   int32_t* counters;
   uint32_t* sync;         // barrier counter, zero at launch
   uint4* phase_table;     // [4 * n_layers][PARAM_QUADS]: every phase's parameters
@@ -166,8 +171,8 @@ __device__ __forceinline__ void stack_store_row(const DmmaParams& p, int R, floa
 // single warp finished.  Warp w's partial of tile t sits in its slot 0 when t
 // is the first tile of its range, else in slot 1.  A tile inside the CTA is
 // summed here in warp order and written; a tile that straddles CTAs leaves
-// the CTA's sum in gp[cta][s] (s = 0 for the CTA's first tile, 1 for its
-// last) for the next phase.  `wbeg` = first unit of each warp of the CTA
+// the CTA's sum in gp[copy][cta][s] (s = 0 for the CTA's first tile, 1 for
+// its last; every copy) for the next phase.  `wbeg` = first unit of each warp of the CTA
 // (17 entries), `wfirst` = first tile of each warp.
 __device__ __forceinline__ void stack_cta_reduce(const DmmaParams& p, const int32_t* wbeg, const int32_t* wfirst,
                                                  const float* wslots, float* gp, int warp, int lane) {
@@ -201,7 +206,9 @@ __device__ __forceinline__ void stack_cta_reduce(const DmmaParams& p, const int3
         // the association of the single-phase kernel: (0 + group sum) + 0
         stack_store_row(p, t * 16 + lane, (0.f + v) + 0.f);
       } else {
-        __stcg(gp + ((size_t)blockIdx.x * 2 + (t == T0 ? 0 : 1)) * 16 + lane, v);
+        const size_t o = ((size_t)blockIdx.x * 2 + (t == T0 ? 0 : 1)) * 16 + lane;
+#pragma unroll
+        for (int r = 0; r < STACK_PART_COPIES; ++r) __stcg(gp + (size_t)r * gridDim.x * 32 + o, v);
       }
     }
   }
@@ -219,6 +226,7 @@ __device__ __forceinline__ void stack_cta_reduce(const DmmaParams& p, const int3
 __device__ __forceinline__ void stack_fixups(const DmmaParams& q, const int2* sent, const float* gq, uint16_t* fixb,
                                              int32_t* tmap, int f, int tid) {
   const int grid = gridDim.x;
+  gq += (size_t)(blockIdx.x % STACK_PART_COPIES) * grid * 32;  // this CTA's copy
   for (int task = tid; task < grid * 2; task += DMMA_THREADS) {  // one pass for grids up to 256 CTAs
     const int c = task >> 1, h = task & 1;                         // rows 8h .. 8h+7 of the tile
     const bool writer = c == (int)blockIdx.x;
@@ -403,7 +411,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
   const int grid_warps = gridDim.x * DMMA_WARPS;
   const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
   const int nphases = 4 * sp.n_layers;
-  const size_t gstride = (size_t)gridDim.x * 32;  // floats of one phase's CTA partials
+  const size_t gstride = (size_t)STACK_PART_COPIES * gridDim.x * 32;  // floats of one phase's CTA partials
   auto slot = [&](int f) -> DmmaParams& { return *reinterpret_cast<DmmaParams*>(slots + (f & 3) * PARAM_QUADS); };
   auto sentf = [&](int f) { return sentt + (f & 1) * gridDim.x; };
   auto wbeg = [&](int f) { return wbegt + (f & 1) * (DMMA_WARPS + 1); };
