@@ -33,6 +33,7 @@ constexpr int UM_STAGES = 4;
 constexpr int UM_DEC_THREADS = 256;             // 8 decoder warps: 2 threads per row
 constexpr int UM_THREADS = 128 + UM_DEC_THREADS;
 constexpr int UM_TIMEOUT_STATUS = 7;  // TQ_ERR_TIMEOUT
+constexpr int UM_SPLIT_BATCH = 4;     // split partials loaded together in the split-k sum
 
 struct UmmaParams {
   CUtensorMap tmap_x;         // x' fp16 [m][k]: box {64, BN}, 128B swizzle
@@ -355,20 +356,28 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
           float4 acc[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int sp = 0; sp < p.splits; ++sp) {
-            float4 v4[4];
+          // the loads of up to UM_SPLIT_BATCH splits are all in flight before
+          // the first add (the sum is latency-bound otherwise)
+          for (int sp0 = 0; sp0 < p.splits; sp0 += UM_SPLIT_BATCH) {
+            float4 v4[UM_SPLIT_BATCH][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int i = i0 + u * UM_DEC_THREADS;
-              v4[u] = i < Q ? __ldcg(tp + (size_t)sp * Q + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+            for (int b = 0; b < UM_SPLIT_BATCH; ++b)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              acc[u].x += v4[u].x;
-              acc[u].y += v4[u].y;
-              acc[u].z += v4[u].z;
-              acc[u].w += v4[u].w;
-            }
+              for (int u = 0; u < 4; ++u) {
+                const int i = i0 + u * UM_DEC_THREADS;
+                v4[b][u] = (i < Q && sp0 + b < p.splits) ? __ldcg(tp + (size_t)(sp0 + b) * Q + i)
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+#pragma unroll
+            for (int b = 0; b < UM_SPLIT_BATCH; ++b)
+              if (sp0 + b < p.splits)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  acc[u].x += v4[b][u].x;
+                  acc[u].y += v4[b][u].y;
+                  acc[u].z += v4[b][u].z;
+                  acc[u].w += v4[b][u].w;
+                }
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
