@@ -24,7 +24,7 @@ OPS = ("q", "k", "v", "o", "gate", "up", "down")
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
            "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
-           "tq_layer_stack_buffers")
+           "tq_layer_stack_buffers", "tq_layer_stack_outputs")
 
 
 class TqError(RuntimeError):
@@ -81,6 +81,7 @@ def _lib():
             "tq_layer_phase": ([LY, i32, vp, i32, u64, vp, vp, vp, sz, vp], ctypes.c_int),
             "tq_layer_stack": ([LY, i32, vp, i32, u64, vp, vp, sz, vp], ctypes.c_int),
             "tq_layer_stack_buffers": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "tq_layer_stack_outputs": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "tq_last_cuda_error": ([], ctypes.c_int),
         }
@@ -246,6 +247,15 @@ def tq_layer_stack_buffers(layers, m: int):
     arr = (tq_layer_t * len(layers))(*layers)
     out = (ctypes.c_size_t * 5)()
     _ok(_lib().tq_layer_stack_buffers(arr, len(layers), m, out), "tq_layer_stack_buffers")
+    return list(out)
+
+
+def tq_layer_stack_outputs(layers, m: int):
+    """Workspace byte offsets of the fp32 outputs of the last layer's four
+    phases (equal offsets when m > 1: only the last phase's survive)."""
+    arr = (tq_layer_t * len(layers))(*layers)
+    out = (ctypes.c_size_t * 4)()
+    _ok(_lib().tq_layer_stack_outputs(arr, len(layers), m, out), "tq_layer_stack_outputs")
     return list(out)
 
 

@@ -695,6 +695,15 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
   return TQ_OK;
 }
 
+// Output regions of the four phase types: at m == 1 one each, down first (at
+// L.y), then q|k|v, o, gate|up; at m > 1 one shared region.
+static size_t stack_y_offset(const StackWs& L, int32_t m, int phase) {
+  if (m != 1) return L.y;
+  const size_t yb = (L.a - L.y) / 4;
+  const int order[4] = {1, 2, 3, 0};
+  return L.y + order[phase] * yb;
+}
+
 // The whole batch-1 stack as one cooperative persistent kernel.  Returns
 // TQ_ERR_SHAPE (and launches nothing) when the stack does not qualify: more
 // than STACK_MAX_LAYERS layers, phases with different codebooks, or a phase
@@ -743,11 +752,7 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.buf[1] = reinterpret_cast<uint16_t*>(ws + L.b);
   sp.buf[2] = reinterpret_cast<uint16_t*>(ws + L.c);
   sp.buf[3] = reinterpret_cast<uint16_t*>(ws + L.h);
-  {
-    const size_t yb = (L.a - L.y) / 4;  // one region per phase type: down, qkv, o, gate|up
-    const int order[4] = {1, 2, 3, 0};
-    for (int ph = 0; ph < 4; ++ph) sp.y[ph] = reinterpret_cast<float*>(ws + L.y + order[ph] * yb);
-  }
+  for (int ph = 0; ph < 4; ++ph) sp.y[ph] = reinterpret_cast<float*>(ws + stack_y_offset(L, 1, ph));
   sp.signs = reinterpret_cast<uint32_t*>(ws + L.signs);
   sp.sign_words = L.sign_words;
   sp.seed = seed;
@@ -799,6 +804,15 @@ int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, int32_t m
   return TQ_OK;
 }
 
+int tq_layer_stack_outputs(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[4]) {
+  if (!offsets) return TQ_ERR_NULL;
+  StackWs L;
+  int st = stack_layout(layers, n_layers, m, &L);
+  if (st != TQ_OK) return st;
+  for (int p = 0; p < 4; ++p) offsets[p] = stack_y_offset(L, m, p);
+  return TQ_OK;
+}
+
 int tq_layer_stack_workspace(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t* bytes) {
   if (!bytes) return TQ_ERR_NULL;
   StackWs L;
@@ -821,7 +835,6 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
   st = check_arch(&sms);
   if (st != TQ_OK) return st;
   char* ws = static_cast<char*>(workspace_d);
-  float* y = reinterpret_cast<float*>(ws + L.y);
   uint16_t* a = reinterpret_cast<uint16_t*>(ws + L.a);
   uint16_t* b = reinterpret_cast<uint16_t*>(ws + L.b);
   uint16_t* c = reinterpret_cast<uint16_t*>(ws + L.c);
@@ -838,7 +851,8 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
     const uint16_t* ins[4] = {in0, a, b, c};
     uint16_t* outs[4] = {a, b, c, out3};
     for (int p = 0; p < 4; ++p) {
-      st = run_phase(&layers[l], p, ins[p], m, tq_stack_phase_seed(seed, l, p), y, outs[p], ws, phase_bytes, sms, s);
+      float* yp = reinterpret_cast<float*>(ws + stack_y_offset(L, m, p));
+      st = run_phase(&layers[l], p, ins[p], m, tq_stack_phase_seed(seed, l, p), yp, outs[p], ws, phase_bytes, sms, s);
       if (st != TQ_OK) return st;
     }
   }

@@ -226,6 +226,17 @@ TQ_API int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint
  * buffers are scratch for the next call. */
 TQ_API int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[5]);
 
+/* Byte offsets, inside a tq_layer_stack workspace for these layers and m, of
+ * the fp32 outputs y [m][n_phase] of the last layer's four phases (q|k|v,
+ * o, gate|up, down: every op of the phase, concatenated by rows) when
+ * tq_layer_stack has returned.  At m == 1 each phase has its own buffer; at
+ * m > 1 the phases share one buffer (all four offsets are equal) and only
+ * the last phase's outputs are left in it.  offsets[3] equals
+ * tq_layer_stack_buffers' offsets[4].  For inspection and tests; the
+ * pages define no such query.  TQ_ERR_NULL / TQ_ERR_SHAPE as
+ * tq_layer_stack_workspace. */
+TQ_API int tq_layer_stack_outputs(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[4]);
+
 /* Human-readable text of a status code (static storage). */
 TQ_API const char* tq_status_string(int status);
 

@@ -60,6 +60,31 @@ def test_stack_workspace_sizes_monotone():
         tq.tq_gemm_workspace(1024, 1024, 5000)
 
 
+def _fake_layer(hidden, q, kv, inter):
+    """A tq_layer_t of fake (aligned, never dereferenced) pointers."""
+    def w(n, k):
+        return tq.tq_weight_t(16, 16, 16, n, k)
+    return tq.tq_layer_t(w(q, hidden), w(kv, hidden), w(kv, hidden), w(hidden, q), w(inter, hidden),
+                         w(inter, hidden), w(hidden, inter))
+
+
+def test_stack_output_offsets():
+    """Host-side layout only: per-phase output buffers at batch 1, one shared
+    buffer otherwise; the down outputs are where tq_layer_stack_buffers says."""
+    layers = [_fake_layer(1024, 1536, 200, 2560)] * 3
+    o1 = tq.tq_layer_stack_outputs(layers, 1)
+    assert len(set(o1)) == 4 and all(o % 256 == 0 for o in o1)
+    assert o1[3] == tq.tq_layer_stack_buffers(layers, 1)[4]
+    # each buffer holds the widest phase (gate|up: 2 x 2560 fp32 rows) without overlap
+    sizes = sorted(o1)
+    assert all(b - a >= 4 * 2 * 2560 for a, b in zip(sizes, sizes[1:]))
+    assert max(o1) + 4 * 2 * 2560 <= tq.tq_layer_stack_workspace(layers, 1)
+    o4 = tq.tq_layer_stack_outputs(layers, 4)
+    assert len(set(o4)) == 1 and o4[0] == tq.tq_layer_stack_buffers(layers, 4)[4]
+    with pytest.raises(tq.TqError):
+        tq.tq_layer_stack_outputs([_fake_layer(1024, 1536, 200, 2000)], 1)  # gate.n not a multiple of 512
+
+
 def test_argument_checks_before_any_device_call():
     L = tq.lib()
     W = tq.tq_weight_t(16, 16, 16, 32, 512)  # fake, aligned addresses; never dereferenced
