@@ -212,36 +212,47 @@ def run_reference(args, shape, m):
 # ---- our arm ------------------------------------------------------------------------
 
 def cpu_baseline_quick(shape, m):
-    """The oracle on ~10-20 s of host work: a row sample of layer 0."""
+    """The oracle on ~10-20 s of host work: the same fraction of the rows of
+    each op of layer 0 (with its RHT), each op's time scaled by its row count,
+    summed, and scaled to the whole stack."""
     import oracle
     oracle.build()
     seed = 0
     cb = tqsynth.codebook(seed)
     ops = shape.ops()
     t_target = 12.0
-    t0 = time.perf_counter()
+    cost = []  # seconds per row of each op (2-row probe)
     for i, (op, n, k) in enumerate(ops):
         c = tqsynth.codes_rows(seed, 0, i, k, 0, 2)
         s = tqsynth.scales(seed, 0, i, 2, k)
+        t0 = time.perf_counter()
         oracle.linear_rows(c, s, cb, k, np.zeros((m, k)), m, 0, 2)
-    per_row = (time.perf_counter() - t0) / 2
-    rows = max(1, min(min(n for _, n, _ in ops), int(t_target / max(per_row, 1e-9))))
+        cost.append((time.perf_counter() - t0) / 2)
+    t_est = sum(n * c for (_, n, _), c in zip(ops, cost))  # one whole layer
+    frac = min(1.0, t_target / max(t_est, 1e-9))
+    n_layers = max(1, min(shape.layers, int(round(t_target / max(t_est, 1e-9))))) if frac >= 1.0 else 1
     x = tqsynth.activations(seed, m, shape.hidden)
-    ts = time.perf_counter()
-    done = 0
-    for i, (op, n, k) in enumerate(ops):
-        xin = x if k == shape.hidden else tqsynth.activations(seed + 1 + i, m, k)
-        xr = oracle.rht(xin, m, k, oracle.stack_phase_seed(seed, 0, 0))
-        c = tqsynth.codes_rows(seed, 0, i, k, 0, rows)
-        s = tqsynth.scales(seed, 0, i, rows, k)
-        oracle.linear_rows(c, s, cb, k, xr, m, 0, rows)
-        done += rows
-    t = time.perf_counter() - ts
+    t_layers, t_all, done = 0.0, 0.0, 0
+    for l in range(n_layers):
+        for i, (op, n, k) in enumerate(ops):
+            rows = max(1, min(n, int(round(frac * n))))
+            xin = x if k == shape.hidden else tqsynth.activations(seed + 1 + i, m, k)
+            c = tqsynth.codes_rows(seed, l, i, k, 0, rows)
+            s = tqsynth.scales(seed, l, i, rows, k)
+            ts = time.perf_counter()
+            xr = oracle.rht(xin, m, k, oracle.stack_phase_seed(seed, l, 0))
+            oracle.linear_rows(c, s, cb, k, xr, m, 0, rows)
+            t = time.perf_counter() - ts
+            t_all += t
+            t_layers += t * n / rows
+            done += rows
     full_rows = sum(n for _, n, _ in ops)
-    t_token = t * (full_rows / done) * shape.layers / m
+    t_token = t_layers / n_layers * shape.layers / m
+    what = (f"all {full_rows} rows of layers 0-{n_layers - 1}" if frac >= 1.0 else
+            f"{done} of the {full_rows} rows of layer 0 (the same fraction of each of its 7 ops)")
     return {"value": 1.0 / t_token, "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": f"{rows} rows of each of the 7 ops of layer 0 ({done} of {full_rows} rows) with their RHTs, "
-                      f"m={m}, {t:.1f} s single-threaded, scaled to {shape.layers} layers"}
+            "sample": f"{what} with their RHTs, m={m}, {t_all:.1f} s single-threaded, each op scaled by its "
+                      f"row count, then to {shape.layers} layers"}
 
 
 def main():
