@@ -95,10 +95,9 @@ size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 int dmma_nt_for(int32_t m) {
   if (m <= 8) return 1;
   if (m <= 16) return 2;
-  if (m <= 32) return 4;
-  return 8;
+  return 4;
 }
-constexpr int kDmmaMaxM = 64;  // one dmma launch covers up to 64 tokens
+constexpr int kDmmaMaxM = 32;  // one dmma launch covers up to 32 tokens (4 column tiles)
 
 struct DmmaWs {
   size_t counters_off, partials_off, bytes;
@@ -168,7 +167,7 @@ int dmma_launch_lv(DmmaParams& p, int lv, int num_sms, cudaStream_t stream) {
   }
 }
 
-// Fill the shape / workspace fields of p and launch.  p.m <= 64.
+// Fill the shape / workspace fields of p and launch.  p.m <= 32.
 int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
   const int nt = hilo ? 1 : dmma_nt_for(p.m);
   const int mc = hilo ? 1 : nt * 8;
@@ -187,8 +186,7 @@ int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, c
   switch (nt) {
     case 1: return dmma_launch_lv<1, false>(p, lv, num_sms, stream);
     case 2: return dmma_launch_lv<2, false>(p, lv, num_sms, stream);
-    case 4: return dmma_launch_lv<4, false>(p, lv, num_sms, stream);
-    default: return dmma_launch_lv<8, false>(p, lv, num_sms, stream);
+    default: return dmma_launch_lv<4, false>(p, lv, num_sms, stream);
   }
 }
 

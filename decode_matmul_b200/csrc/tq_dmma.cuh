@@ -424,9 +424,10 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
 
     const uint8_t* xs_lane = xs + (((b << 4) << 2) + q) * 16 + (g & 1) * 8;
     const uint16_t* xg_lane[NT];
+    uint4 bpair[NT];
 #pragma unroll
     for (int jt = 0; jt < NT; ++jt)
-      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + (size_t)b * 256 + q * 4;
+      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + (size_t)b * 256 + q * 8;
     // previous code byte of each row chunk (state of code 0); 0 at a block start
     uint32_t pa = __shfl_up_sync(0xffffffffu, cur.ca.w, 1) >> 24;
     uint32_t pb = __shfl_up_sync(0xffffffffu, cur.cb.w, 1) >> 24;
@@ -459,10 +460,15 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
           const uint2 bw = lds_b_hilo(xs_lane + j * 64, lane);
           mma_16816((j & 1) ? acc2[0] : acc[0], a, bw.x, bw.y);
         } else {
+          // one 16-byte load holds this lane's quads of steps j and j + 1
+          if ((j & 1) == 0) {
+#pragma unroll
+            for (int jt = 0; jt < NT; ++jt) bpair[jt] = __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j));
+          }
 #pragma unroll
           for (int jt = 0; jt < NT; ++jt) {
-            const uint2 bv = __ldg(reinterpret_cast<const uint2*>(xg_lane[jt] + 16 * j));
-            mma_16816((j & 1) ? acc2[jt] : acc[jt], a, bv.x, bv.y);
+            const uint32_t b0 = (j & 1) ? bpair[jt].z : bpair[jt].x, b1 = (j & 1) ? bpair[jt].w : bpair[jt].y;
+            mma_16816((j & 1) ? acc2[jt] : acc[jt], a, b0, b1);
           }
         }
       }

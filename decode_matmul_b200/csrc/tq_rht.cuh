@@ -68,12 +68,14 @@ __device__ __forceinline__ void rht512_warp(const uint16_t* __restrict__ x_row, 
 }
 
 // Position of element k of a row in "fragment order": inside each 256-weight
-// block the 64 groups of 4 are stored step-major, (j, q) for group 16q + j,
-// so that the four quads one MMA step of the small-batch kernel reads (lanes
-// q = 0..3, step j) are 32 contiguous bytes.
+// block the 64 groups of 4 (group 16q + j is read by lanes with q = lane % 4
+// at MMA step j of the small-batch kernel) are stored as (j / 2, q, j % 2):
+// a lane's quads of steps j and j + 1 are one 16-byte load, and the four
+// lanes of a step pair read 64 contiguous bytes.
 __host__ __device__ __forceinline__ int frag_pos(int k) {
   const int b = k >> 8, G = (k & 255) >> 2, e = k & 3;
-  return (b << 8) + ((((G & 15) << 2) + (G >> 4)) << 2) + e;
+  const int j = G & 15, q = G >> 4;
+  return (b << 8) + ((((j >> 1) << 3) + (q << 1) + (j & 1)) << 2) + e;
 }
 
 // Standalone RHT: grid-stride over (row, block) warp tasks.  MODE 0: fp32
