@@ -631,12 +631,11 @@ int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf1
 
 // Stack workspace: [phase workspace][y fp32 [m][max n]][a bf16 [m][q]]
 // [b bf16 [m][hidden]][c bf16 [m][inter]][h bf16 [m][hidden]][RHT sign bits]
-// [per-phase parameter and straddling-tile tables (batch-1 persistent
-// kernel)][barrier word]
-constexpr int kStackMaxCtas = 256;  // bound on the persistent stack kernel's grid (tables sized by it)
+// [per-phase parameter table (batch-1 persistent kernel)][barrier word]
+constexpr int kStackMaxCtas = 256;  // bound on the persistent stack kernel's grid
 
 struct StackWs {
-  size_t phase, y, a, b, c, h, signs, params, straddle, sync, total;
+  size_t phase, y, a, b, c, h, signs, params, sync, total;
   uint32_t sign_words;
 };
 
@@ -687,8 +686,7 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
   L->signs = L->h + round_up((size_t)m * hmax * 2, 256);
   L->sign_words = (uint32_t)words;
   L->params = L->signs + round_up((size_t)words * 4, 256);
-  L->straddle = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
-  L->sync = L->straddle + round_up((size_t)n_layers * 4 * kStackMaxCtas * sizeof(int2), 256);
+  L->sync = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
   L->total = L->sync + 256;
   return TQ_OK;
 }
@@ -737,9 +735,8 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   }
   const int lv = dmma_lv_for(true, kmax);
   const size_t smem = (16384u << lv) + (size_t)kmax * 4 + 4 * tq::PARAM_QUADS * 16 +
-                      tq::DMMA_WARPS * 32 * sizeof(float) + (size_t)sms * 16 * sizeof(uint16_t) +
-                      (size_t)kmax / 16 * sizeof(int32_t) + 2 * (size_t)sms * 2 * sizeof(int32_t) +
-                      4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) + 32;
+                      tq::DMMA_WARPS * 32 * sizeof(float) + 4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) +
+                      (size_t)kmax / 512 * sizeof(int32_t) + 32;
   if (smem > 227 * 1024) return TQ_ERR_SHAPE;
   sp.n_layers = n_layers;
   sp.lv = lv;
@@ -759,7 +756,6 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.partials = reinterpret_cast<float*>(ws + kCounterBytes);
   sp.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
   sp.phase_table = reinterpret_cast<uint4*>(ws + L.params);
-  sp.straddle_table = reinterpret_cast<int2*>(ws + L.straddle);
   sp.spin_limit = 1u << 24;  // x 64 ns sleeps: ~1 s, far above any healthy phase
   void (*kern)(tq::StackParams);
   switch (lv) {

@@ -383,9 +383,32 @@ __device__ __forceinline__ uint2 lds_b_hilo(const uint8_t* addr, int lane) {
 // are not published through global memory: their partial sums go to this
 // warp's two shared-memory slots ([2][16] floats, slot 0 = the range's first
 // tile), for a reduction by the whole CTA.
+// With `xflag` (batch 1, persistent stack) the activations are produced
+// block by block while the units run: before reading the x' of a 512-block
+// for the first time, the warp waits (bounded; on timeout the status word
+// gets TQ_ERR_TIMEOUT) until xflag[block] == xtag.
+__device__ __forceinline__ void wait_xflag(const volatile int* xflag, int blk, int xtag, int32_t* status,
+                                           uint32_t spin_limit) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
+    uint32_t spins = 0;
+    while (xflag[blk] != xtag) {
+      if (++spins > spin_limit) {
+        if (status) atomicExch(status, 7);  // TQ_ERR_TIMEOUT
+        break;
+      }
+      __nanosleep(20);
+    }
+  }
+  __syncwarp();
+  __threadfence_block();
+}
+
 template <int LV, int NT, bool HILO>
 __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* smem, const uint8_t* xs, int64_t W,
-                                           DmmaCursor& c, int lane, float* wslots = nullptr) {
+                                           DmmaCursor& c, int lane, float* wslots = nullptr,
+                                           const volatile int* xflag = nullptr, int xtag = 0,
+                                           int32_t* status = nullptr, uint32_t spin_limit = 0) {
   constexpr int V = 1 << LV;
   constexpr int SH = 3 + LV;
   const int g = lane >> 2, q = lane & 3;
@@ -402,6 +425,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
     for (int i = 0; i < 4; ++i) acc[jt][i] = acc2[jt][i] = 0.f;
 
   const int nunits = (int)(c.we - c.wb);
+  int ready_rb = -1;  // x' block known to be stored (xflag mode)
   bool has_head = false, has_tail = false;
   int head_t = 0, tail_t = 0;
   float hacc[NT][4];
@@ -422,6 +446,10 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
       nxt = dmma_fetch(nrows, bn);
     }
 
+    if (HILO && xflag && (b >> 1) != ready_rb) {
+      ready_rb = b >> 1;
+      wait_xflag(xflag, ready_rb, xtag, status, spin_limit);
+    }
     const uint8_t* xs_lane = xs + (((b << 4) << 2) + q) * 16 + (g & 1) * 8;
     const uint16_t* xg_lane[NT];
     uint4 bpair[NT];

@@ -61,7 +61,6 @@ struct StackParams {
   int32_t* counters;
   uint32_t* sync;         // barrier counter, zero at launch
   uint4* phase_table;     // [4 * n_layers][PARAM_QUADS]: every phase's parameters
-  int2* straddle_table;   // [4 * n_layers][grid]: every phase's straddling-tile entries
   int32_t* status;
   uint32_t spin_limit;
 };
@@ -214,66 +213,71 @@ __device__ __forceinline__ void stack_cta_reduce(const DmmaParams& p, const int3
   }
 }
 
-// The previous phase's tiles (parameters q, CTA partials gq) that straddle
-// CTAs.  Tile T is taken once, under the CTA c where it starts (T is then the
-// last tile of c's range): sent[c] = {T, cz | s0 << 16} (T < 0: none), with
-// cz the last contributing CTA and s0 the slot of c's partial.  Its value is
-// the sum over the contributing CTAs c .. cz in order.  Rows of the consumed
-// op (the handoff) go, rounded as the handoff is, to fixb[c][16] with
-// tmap[T] = f << 16 | c, for the RHT of this phase; CTA c alone writes the
-// outputs (y, handoff) of entry c.  With fixb == nullptr only those writes
-// are done.
-__device__ __forceinline__ void stack_fixups(const DmmaParams& q, const int2* sent, const float* gq, uint16_t* fixb,
-                                             int32_t* tmap, int f, int tid) {
-  const int grid = gridDim.x;
-  gq += (size_t)(blockIdx.x % STACK_PART_COPIES) * grid * 32;  // this CTA's copy
-  for (int task = tid; task < grid * 2; task += DMMA_THREADS) {  // one pass for grids up to 256 CTAs
-    const int c = task >> 1, h = task & 1;                         // rows 8h .. 8h+7 of the tile
-    const bool writer = c == (int)blockIdx.x;
-    if (!fixb && !writer) continue;
-    const int2 e = sent[c];
-    if (e.x < 0) continue;
-    const int T = e.x, cz = e.y & 0xFFFF, s0 = e.y >> 16;
-    const bool consumed = fixb && T * 16 < q.handoff_rows;
-    if (!consumed && !writer) continue;
-    float4 v[4][2];
+// Tile T of phase q (units T*B .. T*B+B-1) straddles CTAs when its first and
+// last units belong to different CTAs ca < cz; s0 is the slot of ca's partial
+// (0 when T is the first tile of ca's range).
+__device__ __forceinline__ bool sk_straddle(const DmmaParams& q, int T, int& ca, int& cz, int& s0) {
+  const int64_t t0 = (int64_t)T * q.blocks, t1 = t0 + q.blocks;
+  ca = sk_cta_of(q, t0);
+  cz = sk_cta_of(q, t1 - 1);
+  if (ca == cz) return false;
+  s0 = sk_cta_begin(q, ca) >= t0 ? 0 : 1;
+  return true;
+}
+
+// Rows i0 .. i0+n-1 (n = 16 or 8) of a straddling tile: the sum of its CTA
+// partials (gq = this CTA's copy) in CTA order, with the association of the
+// single-phase kernel's last-arriver sum ((0 + group sums) + 0).  Two
+// contributors' loads are in flight together.
+template <int N>
+__device__ __forceinline__ void sk_sum_rows(const float* gq, int ca, int cz, int s0, int i0, float (&v)[N]) {
+  static_assert(N % 4 == 0, "rows in float4s");
+  float4 a[2][N / 4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4* src = reinterpret_cast<const float4*>(gq + ((size_t)(c + i) * 2 + (i ? 0 : s0)) * 16) + 2 * h;
-      const bool live = c + i <= cz;
-      v[i][0] = live ? __ldcg(src) : make_float4(0.f, 0.f, 0.f, 0.f);
-      v[i][1] = live ? __ldcg(src + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float acc[8];
+  for (int i = 0; i < 2; ++i) {
+    const float4* src = reinterpret_cast<const float4*>(gq + ((size_t)(ca + i) * 2 + (i ? 0 : s0)) * 16 + i0);
 #pragma unroll
-    for (int e8 = 0; e8 < 8; ++e8) acc[e8] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (c + i <= cz) {
-        const float* vv = reinterpret_cast<const float*>(&v[i][0]);
-#pragma unroll
-        for (int e8 = 0; e8 < 8; ++e8) acc[e8] += vv[e8];
-      }
-    for (int cc = c + 4; cc <= cz; ++cc) {  // a tile over more than four CTAs
-      const float4* src = reinterpret_cast<const float4*>(gq + (size_t)cc * 2 * 16) + 2 * h;
-      const float4 u0 = __ldcg(src), u1 = __ldcg(src + 1);
-      acc[0] += u0.x;
-      acc[1] += u0.y;
-      acc[2] += u0.z;
-      acc[3] += u0.w;
-      acc[4] += u1.x;
-      acc[5] += u1.y;
-      acc[6] += u1.z;
-      acc[7] += u1.w;
-    }
-#pragma unroll
-    for (int e8 = 0; e8 < 8; ++e8) {
-      const float fin = acc[e8] + 0.f;
-      if (consumed) fixb[c * 16 + h * 8 + e8] = f_to_bf16_bits(q.alpha * fin);
-      if (writer) stack_store_row(q, T * 16 + h * 8 + e8, fin);
-    }
-    if (consumed && h == 0) tmap[T] = (f << 16) | c;
+    for (int u = 0; u < N / 4; ++u) a[i][u] = (ca + i <= cz) ? __ldcg(src + u) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+#pragma unroll
+  for (int e = 0; e < N; ++e) v[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (ca + i <= cz) {
+      const float* aa = reinterpret_cast<const float*>(&a[i][0]);
+#pragma unroll
+      for (int e = 0; e < N; ++e) v[e] += aa[e];
+    }
+  for (int cc = ca + 2; cc <= cz; ++cc) {  // a tile over more than two CTAs
+    const float4* src = reinterpret_cast<const float4*>(gq + (size_t)cc * 2 * 16 + i0);
+#pragma unroll
+    for (int u = 0; u < N / 4; ++u) {
+      const float4 w = __ldcg(src + u);
+      v[4 * u] += w.x;
+      v[4 * u + 1] += w.y;
+      v[4 * u + 2] += w.z;
+      v[4 * u + 3] += w.w;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < N; ++e) v[e] = v[e] + 0.f;
+}
+
+// The outputs (y, handoff) of the straddling tile of phase q that starts in
+// this CTA's range, if any; lanes 0-3, four rows each.  Every such tile
+// starts in exactly one CTA, so each is written once.
+__device__ __forceinline__ void stack_own_straddle(const DmmaParams& q, const float* gq, int tid) {
+  if (tid >= 4) return;
+  const int64_t B = q.blocks;
+  const int64_t b0 = sk_cta_begin(q, blockIdx.x), b1 = sk_cta_begin(q, blockIdx.x + 1);
+  if (b0 >= b1) return;
+  const int T = (int)((b1 - 1) / B);
+  const int64_t t0 = (int64_t)T * B, t1 = t0 + B;
+  if (t0 < b0 || t1 <= b1) return;  // starts in an earlier CTA, or ends inside this one
+  const int cz = sk_cta_of(q, t1 - 1);
+  float v[4];
+  sk_sum_rows<4>(gq, blockIdx.x, cz, (b0 / B == T) ? 0 : 1, tid * 4, v);
+  for (int e = 0; e < 4; ++e) stack_store_row(q, T * 16 + tid * 4 + e, v[e]);
 }
 
 // RHT of one 512-block with the diagonal taken from the sign table, in two
@@ -297,19 +301,24 @@ __device__ __forceinline__ RhtIn rht_table_load(const uint16_t* x, int blk, cons
   return r;
 }
 
-// Transform block blk and store it as hi/lo quads.  When tmap marks this
-// lane's 16 inputs (one tile of the previous phase) as summed in this phase,
-// they come from fixb instead of the handoff in global memory.
-__device__ __forceinline__ void rht_table_finish(RhtIn r, int blk, const uint16_t* fixb, const int32_t* tmap, int f,
-                                                 uint8_t* xs) {
+// Transform block blk and store it as hi/lo quads, then mark the block ready
+// for this CTA's unit loops (xflag[blk] = tag).  With q, a lane whose 16
+// inputs (tile 32 blk + lane of phase q) straddle CTAs sums them from the CTA
+// partials gq and rounds them as the handoff is, instead of the handoff value
+// in global memory (written by its own CTA only after this phase's barrier).
+__device__ __forceinline__ void rht_block(RhtIn r, int blk, const DmmaParams* q, const float* gq, uint8_t* xs,
+                                          volatile int* xflag, int tag) {
   const int lane = threadIdx.x & 31;
-  if (tmap) {
-    const int32_t tg = tmap[blk * 32 + lane];
-    if ((tg >> 16) == f) {
-      const uint4* src = reinterpret_cast<const uint4*>(fixb + (tg & 0xFFFF) * 16);
-      r.p0 = src[0];
-      r.p1 = src[1];
-    }
+  int ca, cz, s0;
+  if (q && sk_straddle(*q, blk * 32 + lane, ca, cz, s0)) {
+    float v[16];
+    sk_sum_rows<16>(gq, ca, cz, s0, 0, v);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i] = f_to_bf16_bits(q->alpha * v[2 * i]) | (f_to_bf16_bits(q->alpha * v[2 * i + 1]) << 16);
+    r.p0 = make_uint4(w[0], w[1], w[2], w[3]);
+    r.p1 = make_uint4(w[4], w[5], w[6], w[7]);
   }
   const uint32_t w[8] = {r.p0.x, r.p0.y, r.p0.z, r.p0.w, r.p1.x, r.p1.y, r.p1.z, r.p1.w};
   float v[16];
@@ -325,46 +334,27 @@ __device__ __forceinline__ void rht_table_finish(RhtIn r, int blk, const uint16_
 #pragma unroll
   for (int r4 = 0; r4 < 4; ++r4)
     store_hilo(xs, blk * 128 + lane * 4 + r4, v[4 * r4], v[4 * r4 + 1], v[4 * r4 + 2], v[4 * r4 + 3]);
+  __syncwarp();
+  __threadfence_block();
+  if (lane == 0) xflag[blk] = tag;
 }
 
-// The phase's activations x' = RHT(x) as hi/lo fp16 quads in shared memory.
-// Block blk goes to warp blk % 16 and up to three blocks per warp have their
-// loads in flight together; meanwhile the CTA sums the previous phase's
-// straddling tiles (q != nullptr, entries sentq) and then fills the next
-// phase's warp tables (pn != nullptr).  Ends with a __syncthreads.
-__device__ __forceinline__ void stack_warp_tables(const DmmaParams& p, int32_t* wbeg, int32_t* wfirst, int tid);
-
-__device__ __forceinline__ void stack_rht(const DmmaParams& p, const DmmaParams* q, const int2* sentq, const float* gq,
-                                          const uint32_t* signs, uint8_t* xs, uint16_t* fixb, int32_t* tmap, int f,
-                                          int tid, const DmmaParams* pn, int32_t* wbegn, int32_t* wfirstn) {
-  const int warp = tid >> 5;
+// This warp's share of the phase's activations x' = RHT(x): blocks warp,
+// warp + 16, ...; the loads of up to three blocks are in flight together.
+// No CTA-wide synchronisation: each block is flagged when it is stored.
+__device__ __forceinline__ void stack_rht(const DmmaParams& p, const DmmaParams* q, const float* gq,
+                                          const uint32_t* signs, uint8_t* xs, volatile int* xflag, int tag,
+                                          int warp) {
   const int nb = p.k / 512;
   RhtIn in[3];
 #pragma unroll
   for (int r = 0; r < 3; ++r)
     if (warp + DMMA_WARPS * r < nb) in[r] = rht_table_load(p.x_bf16, warp + DMMA_WARPS * r, signs);
-  if (q) stack_fixups(*q, sentq, gq, fixb, tmap, f, tid);
-  __syncthreads();
-  if (pn) stack_warp_tables(*pn, wbegn, wfirstn, tid);  // the next phase's
-  const int32_t* tm = q ? tmap : nullptr;
 #pragma unroll
   for (int r = 0; r < 3; ++r)
-    if (warp + DMMA_WARPS * r < nb) rht_table_finish(in[r], warp + DMMA_WARPS * r, fixb, tm, f, xs);
+    if (warp + DMMA_WARPS * r < nb) rht_block(in[r], warp + DMMA_WARPS * r, q, gq, xs, xflag, tag);
   for (int blk = warp + 3 * DMMA_WARPS; blk < nb; blk += DMMA_WARPS)  // k > 24576 only
-    rht_table_finish(rht_table_load(p.x_bf16, blk, signs), blk, fixb, tm, f, xs);
-  __syncthreads();
-}
-
-// The straddling tile entered under CTA c in phase p (see stack_fixups).
-__device__ __forceinline__ int2 stack_straddle_entry(const DmmaParams& p, int c) {
-  const int64_t B = p.blocks;
-  const int64_t b0 = sk_cta_begin(p, c), b1 = sk_cta_begin(p, c + 1);
-  int2 e = make_int2(-1, 0);
-  if (b0 < b1) {
-    const int64_t T = (b1 - 1) / B, t0 = T * B, t1 = t0 + B;
-    if (t0 >= b0 && t1 > b1) e = make_int2((int)T, sk_cta_of(p, t1 - 1) | ((b0 / B == T) ? 0 : 1) << 16);
-  }
-  return e;
+    rht_block(rht_table_load(p.x_bf16, blk, signs), blk, q, gq, xs, xflag, tag);
 }
 
 // First unit and first tile of each warp of this CTA in phase p.
@@ -400,29 +390,30 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     for (int ph = 0; ph < 4; ++ph) kmax = max(kmax, sp.layers[l].k[ph]);
   // four parameter slots: previous, running, next and next-but-one phase
   uint4* slots = reinterpret_cast<uint4*>(xs + (size_t)kmax * 4);
-  float* wslots = reinterpret_cast<float*>(slots + 4 * PARAM_QUADS);      // [warp][2][16]
-  uint16_t* fixb = reinterpret_cast<uint16_t*>(wslots + DMMA_WARPS * 32);  // [grid][16]
-  int32_t* tmap = reinterpret_cast<int32_t*>(fixb + gridDim.x * 16);       // [kmax / 16]
-  int2* sentt = reinterpret_cast<int2*>(tmap + kmax / 16);                 // [2][grid]
-  int32_t* wbegt = reinterpret_cast<int32_t*>(sentt + 2 * gridDim.x);      // [2][DMMA_WARPS + 1]
-  int32_t* wfirstt = wbegt + 2 * (DMMA_WARPS + 1);                         // [2][DMMA_WARPS + 1]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(wfirstt + 2 * (DMMA_WARPS + 1));
+  float* wslots = reinterpret_cast<float*>(slots + 4 * PARAM_QUADS);       // [warp][2][16]
+  int32_t* wbegt = reinterpret_cast<int32_t*>(wslots + DMMA_WARPS * 32);    // [2][DMMA_WARPS + 1]
+  int32_t* wfirstt = wbegt + 2 * (DMMA_WARPS + 1);                          // [2][DMMA_WARPS + 1]
+  volatile int* xflag = reinterpret_cast<volatile int*>(wfirstt + 2 * (DMMA_WARPS + 1));  // [kmax / 512]
+  volatile int* abort_flag = xflag + kmax / 512;
+  int* duty = const_cast<int*>(abort_flag + 1);  // last phase whose straddle duty was taken
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int grid_warps = gridDim.x * DMMA_WARPS;
   const int64_t W = (int64_t)blockIdx.x * DMMA_WARPS + warp;
   const int nphases = 4 * sp.n_layers;
   const size_t gstride = (size_t)STACK_PART_COPIES * gridDim.x * 32;  // floats of one phase's CTA partials
+  const size_t gcopy = (size_t)(blockIdx.x % STACK_PART_COPIES) * gridDim.x * 32;  // this CTA's copy
   auto slot = [&](int f) -> DmmaParams& { return *reinterpret_cast<DmmaParams*>(slots + (f & 3) * PARAM_QUADS); };
-  auto sentf = [&](int f) { return sentt + (f & 1) * gridDim.x; };
   auto wbeg = [&](int f) { return wbegt + (f & 1) * (DMMA_WARPS + 1); };
   auto wfirst = [&](int f) { return wfirstt + (f & 1) * (DMMA_WARPS + 1); };
+  auto parts = [&](int f) { return sp.partials + (size_t)(f % 3) * gstride; };
 
   if (tid == 0) {
     *abort_flag = 0;
+    *duty = 0;
     stack_phase_params(sp, 0, slot(0), grid_warps);
   }
   if (tid == 32 && nphases > 1) stack_phase_params(sp, 1, slot(1), grid_warps);
-  for (int i = tid; i < kmax / 16; i += DMMA_THREADS) tmap[i] = -1;
+  for (int i = tid; i < kmax / 512; i += DMMA_THREADS) xflag[i] = -1;
   // every phase's parameters, one thread each, into the table read later
   for (int f = blockIdx.x * DMMA_THREADS + tid; f < nphases; f += gridDim.x * DMMA_THREADS) {
     DmmaParams pf;
@@ -434,13 +425,6 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
       memcpy(&tail, reinterpret_cast<const uint8_t*>(&pf) + (sizeof(DmmaParams) / 16) * 16, sizeof(DmmaParams) % 16);
       sp.phase_table[(size_t)f * PARAM_QUADS + sizeof(DmmaParams) / 16] = tail;
     }
-  }
-  // every phase's straddling-tile entries, one (phase, CTA) per thread
-  for (int i = blockIdx.x * DMMA_THREADS + tid; i < nphases * (int)gridDim.x; i += gridDim.x * DMMA_THREADS) {
-    const int f = i / gridDim.x;
-    DmmaParams pf;
-    stack_phase_params(sp, f, pf, grid_warps);
-    sp.straddle_table[i] = stack_straddle_entry(pf, i - f * gridDim.x);
   }
   build_views<LV>(smem, sp.codebook, tid, DMMA_THREADS);
 
@@ -457,7 +441,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     for (int i = 0; i < 32; ++i) bits |= (rht_sign_negative(seed_lp, k0 + i) ? 1u : 0u) << i;
     sp.signs[j] = bits;
   }
-  grid_arrive(sp);  // its __syncthreads publishes slot 0 to the CTA
+  grid_arrive(sp);  // its __syncthreads publishes slots 0 and 1 to the CTA
   uint32_t epoch = 1;
 
   // first phase's tables and code chunk, then the barrier
@@ -474,20 +458,24 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     uint4 nq = make_uint4(0u, 0u, 0u, 0u);
     const bool fetch = tid < PARAM_QUADS && f + 2 < nphases;
     if (fetch) nq = __ldcg(sp.phase_table + (size_t)(f + 2) * PARAM_QUADS + tid);
-    const bool next = f + 1 < nphases;
-    // and this phase's straddling entries (read by the next phase's RHT;
-    // the table was written by all CTAs before the first barrier)
-    int2 se = make_int2(-1, 0);
-    if (tid < (int)gridDim.x) se = __ldcg(sp.straddle_table + (size_t)f * gridDim.x + tid);
-    stack_rht(p, f > 0 ? &slot(f - 1) : nullptr, sentf(f - 1), sp.partials + (size_t)((f + 2) % 3) * gstride,
-              sp.signs + sp.layers[l].sign_off[ph], xs, fixb, tmap, f, tid, next ? &slot(f + 1) : nullptr,
-              wbeg(f + 1), wfirst(f + 1));
+    // this warp's blocks of x' (each flagged when stored), then its units,
+    // which wait only for the blocks they read
+    stack_rht(p, f > 0 ? &slot(f - 1) : nullptr, parts(f + 2) + gcopy, sp.signs + sp.layers[l].sign_off[ph], xs,
+              xflag, f, warp);
     if (fetch) slots[((f + 2) & 3) * PARAM_QUADS + tid] = nq;  // slot of phase f-2: no reader left
-    if (tid < (int)gridDim.x) sentf(f)[tid] = se;      // the previous phase's were read above
-    dmma_units<LV, 1, true>(p, smem, xs, W, c, lane, wslots + warp * 32);
+    if (f + 1 < nphases) stack_warp_tables(slot(f + 1), wbeg(f + 1), wfirst(f + 1), tid);  // read after the barrier
+    dmma_units<LV, 1, true>(p, smem, xs, W, c, lane, wslots + warp * 32, xflag, f, sp.status, sp.spin_limit);
+    // the first warp done writes the outputs of the previous phase's
+    // straddling tile that starts in this CTA (its partials stay until phase
+    // f+2 overwrites them), off the critical path of the slowest warp
+    if (f > 0) {
+      int won = 0;
+      if (lane == 0) won = atomicCAS(duty, f - 1, f) == f - 1;
+      if (__shfl_sync(0xffffffffu, won, 0)) stack_own_straddle(slot(f - 1), parts(f - 1) + gcopy, lane);
+    }
     __syncthreads();
-    stack_cta_reduce(p, wbeg(f), wfirst(f), wslots, sp.partials + (size_t)(f % 3) * gstride, warp, lane);
-    grid_arrive(sp);  // its __syncthreads ends every use of the warp tables and slots
+    stack_cta_reduce(p, wbeg(f), wfirst(f), wslots, parts(f), warp, lane);
+    grid_arrive(sp);  // its __syncthreads ends every use of the warp tables, slots and x'
     ++epoch;
     if (f + 1 == nphases) break;
     // next phase: first code chunk before the barrier wait
@@ -496,8 +484,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
   }
   // the last phase's straddling tiles: summed once every CTA partial is in
   if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;
-  stack_fixups(slot(nphases - 1), sentf(nphases - 1),
-               sp.partials + (size_t)((nphases - 1) % 3) * gstride, nullptr, nullptr, nphases, tid);
+  stack_own_straddle(slot(nphases - 1), parts(nphases - 1) + gcopy, tid);
 }
 
 }  // namespace tq
