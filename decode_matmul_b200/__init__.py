@@ -252,7 +252,7 @@ def tq_layer_stack_buffers(layers, m: int):
 
 def tq_layer_stack_outputs(layers, m: int):
     """Workspace byte offsets of the fp32 outputs of the last layer's four
-    phases (equal offsets when m > 1: only the last phase's survive)."""
+    phases (equal offsets when m > 16: only the last phase's survive)."""
     arr = (tq_layer_t * len(layers))(*layers)
     out = (ctypes.c_size_t * 4)()
     _ok(_lib().tq_layer_stack_outputs(arr, len(layers), m, out), "tq_layer_stack_outputs")

@@ -10,6 +10,7 @@
 #include "tq_dmma.cuh"
 #include "tq_rht.cuh"
 #include "tq_stack1.cuh"
+#include "tq_stackn.cuh"
 #include "tq_umma.cuh"
 
 #include <cudaTypedefs.h>
@@ -634,8 +635,10 @@ int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t* x_bf1
 // [per-phase parameter table (batch-1 persistent kernel)][barrier word]
 constexpr int kStackMaxCtas = 256;  // bound on the persistent stack kernel's grid
 
+constexpr int kStackMaxM = 16;  // the persistent stack kernels run batches of 1 .. 16 tokens
+
 struct StackWs {
-  size_t phase, y, a, b, c, h, signs, params, sync, total;
+  size_t phase, y, a, b, c, h, signs, params, xq, sync, total;
   uint32_t sign_words;
 };
 
@@ -670,42 +673,53 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
   if (m == 1) {
     const size_t pk = kCounterBytes + (size_t)tq::DMMA_MAX_WARPS * 2 * 16 * sizeof(float);
     if (phase < pk) phase = pk;
+  } else if (m <= kStackMaxM) {
+    // the small-batch persistent kernel: three phases of CTA partials (two
+    // tiles of 16 rows x 16 tokens per CTA)
+    const size_t pk = kCounterBytes + (size_t)3 * kStackMaxCtas * 2 * 16 * 16 * sizeof(float);
+    if (phase < pk) phase = pk;
+  }
+  int64_t kmax = 0;
+  for (int l = 0; l < n_layers; ++l) {
+    const int64_t ks[4] = {layers[l].q.k, layers[l].o.k, layers[l].gate.k, layers[l].down.k};
+    for (int p = 0; p < 4; ++p) kmax = ks[p] > kmax ? ks[p] : kmax;
   }
   uint64_t words = 0;
   for (int l = 0; l < n_layers; ++l)
     words += ((uint64_t)layers[l].q.k + layers[l].o.k + layers[l].gate.k + layers[l].down.k) / 32;
   L->phase = 0;
   L->y = round_up(phase, 256);
-  // batch 1 (persistent kernel): one output region per phase type, the down
-  // phase's first so that L->y always holds the last phase's outputs
+  // persistent kernels (m <= 16): one output region per phase type, the
+  // down phase's first so that L->y always holds the last phase's outputs
   const size_t yb = round_up((size_t)m * ymax * 4, 256);
-  L->a = L->y + (m == 1 ? 4 : 1) * yb;
+  L->a = L->y + (m <= kStackMaxM ? 4 : 1) * yb;
   L->b = L->a + round_up((size_t)m * amax * 2, 256);
   L->c = L->b + round_up((size_t)m * bmax * 2, 256);
   L->h = L->c + round_up((size_t)m * cmax * 2, 256);
   L->signs = L->h + round_up((size_t)m * hmax * 2, 256);
   L->sign_words = (uint32_t)words;
   L->params = L->signs + round_up((size_t)words * 4, 256);
-  L->sync = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
+  L->xq = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
+  L->sync = L->xq + (m > 1 && m <= kStackMaxM ? round_up((size_t)m * kmax * 2, 256) : 0);
   L->total = L->sync + 256;
   return TQ_OK;
 }
 
-// Output regions of the four phase types: at m == 1 one each, down first (at
-// L.y), then q|k|v, o, gate|up; at m > 1 one shared region.
+// Output regions of the four phase types: at m <= 16 one each, down first (at
+// L.y), then q|k|v, o, gate|up; beyond, one shared region.
 static size_t stack_y_offset(const StackWs& L, int32_t m, int phase) {
-  if (m != 1) return L.y;
+  if (m > kStackMaxM) return L.y;
   const size_t yb = (L.a - L.y) / 4;
   const int order[4] = {1, 2, 3, 0};
   return L.y + order[phase] * yb;
 }
 
-// The whole batch-1 stack as one cooperative persistent kernel.  Returns
-// TQ_ERR_SHAPE (and launches nothing) when the stack does not qualify: more
-// than STACK_MAX_LAYERS layers, phases with different codebooks, or a phase
-// too wide for shared memory.
-static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in, uint64_t seed,
-                      uint16_t* h_out, char* ws, const StackWs& L, int sms, cudaStream_t s) {
+// The whole stack as one cooperative persistent kernel: stack1_kernel at
+// batch 1, stackn_kernel for 2-16 tokens.  Returns TQ_ERR_SHAPE (and launches
+// nothing) when the stack does not qualify: more than STACK_MAX_LAYERS layers,
+// phases with different codebooks, or a phase too wide for shared memory.
+static int stack_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in, int32_t m, uint64_t seed,
+                     uint16_t* h_out, char* ws, const StackWs& L, int sms, cudaStream_t s) {
   if (n_layers > tq::STACK_MAX_LAYERS || sms > kStackMaxCtas) return TQ_ERR_SHAPE;
   static thread_local tq::StackParams sp;  // large (~25 KB): per-thread storage, copied into the launch
   memset(&sp, 0, sizeof(sp));
@@ -733,11 +747,16 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
       if ((nt[ph] + 15) / 16 > kMaxTiles) return TQ_ERR_SHAPE;
     }
   }
-  const int lv = dmma_lv_for(true, kmax);
-  const size_t smem = (16384u << lv) + (size_t)kmax * 4 + 4 * tq::PARAM_QUADS * 16 +
-                      tq::DMMA_WARPS * 32 * sizeof(float) + 4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) +
-                      (size_t)kmax / 512 * sizeof(int32_t) + 32;
+  const int nt = m <= 8 ? 1 : 2;  // 8-token column tiles of the small-batch kernel
+  const int lv = m == 1 ? dmma_lv_for(true, kmax) : 3;
+  const size_t smem = m == 1 ? (16384u << lv) + (size_t)kmax * 4 + 4 * tq::PARAM_QUADS * 16 +
+                                   tq::DMMA_WARPS * 32 * sizeof(float) + 4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) +
+                                   (size_t)kmax / 512 * sizeof(int32_t) + 32
+                             : (16384u << lv) + (size_t)tq::DMMA_WARPS * 2 * 16 * nt * 8 * sizeof(float) +
+                                   4 * tq::PARAM_QUADS * 16 + 4 * (tq::DMMA_WARPS + 1) * sizeof(int32_t) + 32;
   if (smem > 227 * 1024) return TQ_ERR_SHAPE;
+  sp.m = m;
+  sp.xq = m > 1 ? reinterpret_cast<uint16_t*>(ws + L.xq) : nullptr;
   sp.n_layers = n_layers;
   sp.lv = lv;
   sp.codebook = cb;
@@ -747,7 +766,7 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.buf[1] = reinterpret_cast<uint16_t*>(ws + L.b);
   sp.buf[2] = reinterpret_cast<uint16_t*>(ws + L.c);
   sp.buf[3] = reinterpret_cast<uint16_t*>(ws + L.h);
-  for (int ph = 0; ph < 4; ++ph) sp.y[ph] = reinterpret_cast<float*>(ws + stack_y_offset(L, 1, ph));
+  for (int ph = 0; ph < 4; ++ph) sp.y[ph] = reinterpret_cast<float*>(ws + stack_y_offset(L, m, ph));
   sp.signs = reinterpret_cast<uint32_t*>(ws + L.signs);
   sp.sign_words = L.sign_words;
   sp.seed = seed;
@@ -758,18 +777,24 @@ static int stack1_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t
   sp.phase_table = reinterpret_cast<uint4*>(ws + L.params);
   sp.spin_limit = 1u << 24;  // x 64 ns sleeps: ~1 s, far above any healthy phase
   void (*kern)(tq::StackParams);
-  switch (lv) {
-    case 3: kern = tq::stack1_kernel<3>; break;
-    case 2: kern = tq::stack1_kernel<2>; break;
-    case 1: kern = tq::stack1_kernel<1>; break;
-    default: kern = tq::stack1_kernel<0>; break;
+  if (m > 1) {
+    kern = nt == 1 ? tq::stackn_kernel<3, 1> : tq::stackn_kernel<3, 2>;
+  } else {
+    switch (lv) {
+      case 3: kern = tq::stack1_kernel<3>; break;
+      case 2: kern = tq::stack1_kernel<2>; break;
+      case 1: kern = tq::stack1_kernel<1>; break;
+      default: kern = tq::stack1_kernel<0>; break;
+    }
   }
   TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
   int occ = 0;
   TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
   if (occ < 1) return TQ_ERR_SHAPE;
   // partial sums of straddling tiles: three phases x copies x every CTA x two tiles
-  if ((size_t)3 * tq::STACK_PART_COPIES * sms * 2 * 16 * sizeof(float) > L.y - kCounterBytes) return TQ_ERR_SHAPE;
+  const size_t part_bytes = m == 1 ? (size_t)3 * tq::STACK_PART_COPIES * sms * 2 * 16 * sizeof(float)
+                                   : (size_t)3 * sms * 2 * 16 * nt * 8 * sizeof(float);
+  if (part_bytes > L.y - kCounterBytes) return TQ_ERR_SHAPE;
   TQ_CUDA(cudaMemsetAsync(ws + L.sync, 0, 256, s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)sms);
@@ -835,8 +860,8 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
   uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
   const size_t phase_bytes = L.y;
   cudaStream_t s = (cudaStream_t)stream;
-  if (m == 1) {
-    st = stack1_run(layers, n_layers, h_in_bf16_d, seed, h_out_bf16_d, ws, L, sms, s);
+  if (m <= kStackMaxM) {
+    st = stack_run(layers, n_layers, h_in_bf16_d, m, seed, h_out_bf16_d, ws, L, sms, s);
     if (st != TQ_ERR_SHAPE) return st;  // TQ_ERR_SHAPE: not eligible, run phase by phase
   }
   for (int l = 0; l < n_layers; ++l) {

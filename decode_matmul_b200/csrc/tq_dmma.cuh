@@ -404,7 +404,10 @@ __device__ __forceinline__ void wait_xflag(const volatile int* xflag, int blk, i
   __threadfence_block();
 }
 
-template <int LV, int NT, bool HILO>
+// XCG: the small-batch activations were written earlier in the same launch
+// (persistent stack), so they are read through L2 (ld.global.cg) instead of
+// the read-only path.
+template <int LV, int NT, bool HILO, bool XCG = false>
 __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* smem, const uint8_t* xs, int64_t W,
                                            DmmaCursor& c, int lane, float* wslots = nullptr,
                                            const volatile int* xflag = nullptr, int xtag = 0,
@@ -491,7 +494,9 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
           // one 16-byte load holds this lane's quads of steps j and j + 1
           if ((j & 1) == 0) {
 #pragma unroll
-            for (int jt = 0; jt < NT; ++jt) bpair[jt] = __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j));
+            for (int jt = 0; jt < NT; ++jt)
+              bpair[jt] = XCG ? __ldcg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j))
+                              : __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j));
           }
 #pragma unroll
           for (int jt = 0; jt < NT; ++jt) {
@@ -542,16 +547,27 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
   if (has_head || has_tail) {
     // slot 0 holds the range's first tile, slot 1 a later one
     const int tail_slot = (tail_t == (int)(c.wb / p.blocks)) ? 0 : 1;
-    if (HILO && wslots) {
-      if (q == 0) {
-        if (has_head) {
-          wslots[g] = hacc[0][0] + hacc[0][1];
-          wslots[g + 8] = hacc[0][2] + hacc[0][3];
+    if (wslots) {
+      if (HILO) {
+        if (q == 0) {
+          if (has_head) {
+            wslots[g] = hacc[0][0] + hacc[0][1];
+            wslots[g + 8] = hacc[0][2] + hacc[0][3];
+          }
+          if (has_tail) {
+            wslots[tail_slot * 16 + g] = acc[0][0] + acc[0][1];
+            wslots[tail_slot * 16 + g + 8] = acc[0][2] + acc[0][3];
+          }
         }
-        if (has_tail) {
-          wslots[tail_slot * 16 + g] = acc[0][0] + acc[0][1];
-          wslots[tail_slot * 16 + g + 8] = acc[0][2] + acc[0][3];
-        }
+      } else {  // slot layout [16 rows][NT * 8 tokens], as the global partials
+        constexpr int MC = NT * 8;
+#pragma unroll
+        for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (has_head) wslots[partial_index<NT, HILO>(g, q, jt, i)] = hacc[jt][i];
+            if (has_tail) wslots[tail_slot * 16 * MC + partial_index<NT, HILO>(g, q, jt, i)] = acc[jt][i];
+          }
       }
     } else {
       dmma_publish<NT, HILO>(p, W, g, q, has_head, head_t, hacc, has_tail, tail_t, tail_slot, acc);

@@ -59,6 +59,8 @@ struct StackParams {
   uint64_t seed;
   float* partials;        // per-CTA partials of straddling tiles: [3][STACK_PART_COPIES][grid][2][16]
   int32_t* counters;
+  int32_t m;              // tokens (1 for stack1_kernel)
+  uint16_t* xq;           // small batch: x' fp16 [m][k] in fragment order, written each phase
   uint32_t* sync;         // barrier counter, zero at launch
   uint4* phase_table;     // [4 * n_layers][PARAM_QUADS]: every phase's parameters
   int32_t* status;
@@ -90,9 +92,9 @@ __device__ __forceinline__ void stack_phase_params(const StackParams& sp, int f,
   p.codebook = sp.codebook;
   p.n_total = row0;
   p.k = L.k[ph];
-  p.m = 1;
+  p.m = sp.m;
   p.x_f32 = nullptr;
-  p.x_f16 = nullptr;
+  p.x_f16 = sp.xq;
   p.x_bf16 = ph == 0 ? (l == 0 ? sp.h_in : sp.buf[3]) : sp.buf[ph - 1];
   p.rht_seed = 0;
   p.y = sp.y[ph];

@@ -229,8 +229,8 @@ TQ_API int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, in
 /* Byte offsets, inside a tq_layer_stack workspace for these layers and m, of
  * the fp32 outputs y [m][n_phase] of the last layer's four phases (q|k|v,
  * o, gate|up, down: every op of the phase, concatenated by rows) when
- * tq_layer_stack has returned.  At m == 1 each phase has its own buffer; at
- * m > 1 the phases share one buffer (all four offsets are equal) and only
+ * tq_layer_stack has returned.  At m <= 16 each phase has its own buffer;
+ * beyond, the phases share one buffer (all four offsets are equal) and only
  * the last phase's outputs are left in it.  offsets[3] equals
  * tq_layer_stack_buffers' offsets[4].  For inspection and tests; the
  * pages define no such query.  TQ_ERR_NULL / TQ_ERR_SHAPE as

@@ -69,8 +69,9 @@ def _fake_layer(hidden, q, kv, inter):
 
 
 def test_stack_output_offsets():
-    """Host-side layout only: per-phase output buffers at batch 1, one shared
-    buffer otherwise; the down outputs are where tq_layer_stack_buffers says."""
+    """Host-side layout only: per-phase output buffers up to 16 tokens (the
+    persistent kernels), one shared buffer beyond; the down outputs are where
+    tq_layer_stack_buffers says."""
     layers = [_fake_layer(1024, 1536, 200, 2560)] * 3
     o1 = tq.tq_layer_stack_outputs(layers, 1)
     assert len(set(o1)) == 4 and all(o % 256 == 0 for o in o1)
@@ -79,8 +80,10 @@ def test_stack_output_offsets():
     sizes = sorted(o1)
     assert all(b - a >= 4 * 2 * 2560 for a, b in zip(sizes, sizes[1:]))
     assert max(o1) + 4 * 2 * 2560 <= tq.tq_layer_stack_workspace(layers, 1)
-    o4 = tq.tq_layer_stack_outputs(layers, 4)
-    assert len(set(o4)) == 1 and o4[0] == tq.tq_layer_stack_buffers(layers, 4)[4]
+    o4 = tq.tq_layer_stack_outputs(layers, 16)
+    assert len(set(o4)) == 4 and o4[3] == tq.tq_layer_stack_buffers(layers, 16)[4]
+    o32 = tq.tq_layer_stack_outputs(layers, 32)
+    assert len(set(o32)) == 1 and o32[0] == tq.tq_layer_stack_buffers(layers, 32)[4]
     with pytest.raises(tq.TqError):
         tq.tq_layer_stack_outputs([_fake_layer(1024, 1536, 200, 2000)], 1)  # gate.n not a multiple of 512
 

@@ -186,7 +186,7 @@ def test_layer_phases_teacher_forced(tq, torch_cuda, m):
         _check_handoff(from_dev_u16(h), y.cpu().numpy()[:, :n_hand], hand, hl[0][oracle.HANDOFF_OP[p]].k)
 
 
-@pytest.mark.parametrize("m", [1, 3])
+@pytest.mark.parametrize("m", [1, 3, 9, 16])
 def test_layer_stack_is_the_phase_chain(tq, torch_cuda, m):
     import torch
     hl = _host_layers(SMALL)
@@ -215,22 +215,23 @@ def test_layer_stack_is_the_phase_chain(tq, torch_cuda, m):
     assert drift < 0.05, drift
 
 
-# Batch-1 stacks whose tiles straddle many CTAs: ragged k/v outputs (rows not a
-# multiple of 16, never consumed), and a wide down projection (k = 8704 over
-# 512 output rows: each 16-row tile spans about five CTAs of the persistent
-# kernel, more than its four preloaded contributors).
+# Stacks run by the persistent kernels (1-16 tokens) whose tiles straddle many
+# CTAs: ragged k/v outputs (rows not a multiple of 16, never consumed), and a
+# wide down projection (k = 8704 over 512 output rows: each 16-row tile spans
+# about five CTAs, more than the contributors whose loads are issued together).
 RAGGED = tqsynth.StackShape("ragged", 3, 1024, 1536, 200, 2560)
 WIDE = tqsynth.StackShape("wide", 2, 512, 512, 96, 8704)
 
 
+@pytest.mark.parametrize("m", [1, 5, 12])
 @pytest.mark.parametrize("shape", [RAGGED, WIDE], ids=["ragged", "wide"])
-def test_stack_batch1_straddling_tiles(tq, torch_cuda, shape):
+def test_stack_persistent_straddling_tiles(tq, torch_cuda, shape, m):
     import torch
     hl = _host_layers(shape, seed=3)
     dl, structs = _dev_layers(tq, hl)
-    x = to_dev_u16(tqsynth.activations(7, 1, shape.hidden))
-    args = tq.StackArgs(structs, 1)
-    ws = tq.workspace(tq.tq_layer_stack_workspace(structs, 1))
+    x = to_dev_u16(tqsynth.activations(7, m, shape.hidden))
+    args = tq.StackArgs(structs, m)
+    ws = tq.workspace(tq.tq_layer_stack_workspace(structs, m))
     outs = []
     for _ in range(3):  # the persistent kernel is deterministic from run to run
         out = torch.empty_like(x)
@@ -241,12 +242,12 @@ def test_stack_batch1_straddling_tiles(tq, torch_cuda, shape):
     y_stack = ws[off[4]:off[4] + 4 * shape.hidden].view(torch.float32).clone()
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
     # the last layer's outputs of every phase (ragged k / v rows included)
-    yoff = tq.tq_layer_stack_outputs(structs, 1)
+    yoff = tq.tq_layer_stack_outputs(structs, m)
     last = shape.layers - 1
     y_stack = []
     for p in range(4):
         n_phase = sum(hl[last][op].n for op in oracle.PHASES[p])
-        y_stack.append(ws[yoff[p]:yoff[p] + 4 * n_phase].view(torch.float32).clone())
+        y_stack.append(ws[yoff[p]:yoff[p] + 4 * m * n_phase].view(torch.float32).reshape(m, n_phase).clone())
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
     cur = x
     y_chain = []
@@ -254,18 +255,18 @@ def test_stack_batch1_straddling_tiles(tq, torch_cuda, shape):
         for p in range(4):
             n_phase = sum(hl[l][op].n for op in oracle.PHASES[p])
             n_hand = hl[l][oracle.HANDOFF_OP[p]].n
-            y = torch.empty((1, n_phase), dtype=torch.float32, device="cuda")
-            h = torch.empty((1, n_hand), dtype=torch.int16, device="cuda")
-            wsp = tq.workspace(tq.tq_layer_phase_workspace(L, p, 1))
+            y = torch.empty((m, n_phase), dtype=torch.float32, device="cuda")
+            h = torch.empty((m, n_hand), dtype=torch.int16, device="cuda")
+            wsp = tq.workspace(tq.tq_layer_phase_workspace(L, p, m))
             tq.tq_layer_phase(L, p, cur, tq.tq_stack_phase_seed(9, l, p), y, h, wsp)
             cur = h
             if l == last:
-                y_chain.append(y[0])
+                y_chain.append(y)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], cur)
     for p in range(4):
         assert torch.equal(y_stack[p], y_chain[p]), p
-    assert tq.tq_layer_stack_buffers(structs, 1)[4] == yoff[3]
+    assert tq.tq_layer_stack_buffers(structs, m)[4] == yoff[3]
 
 
 def test_workspace_reused_across_shapes(tq, torch_cuda):
