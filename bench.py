@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 import tqsynth  # noqa: E402
 
+PERSISTENT_MAX_M = 16  # tq_layer_stack runs one persistent kernel up to this many tokens
 METRIC = "decode-GEMV compressed-weight GB/s (% of HBM peak); layer-stack tokens/s at batch 1"
 
 WORKLOADS = {
@@ -134,11 +135,12 @@ def phase_bytes(shape, m):
     return out
 
 
-def ncu_traffic(layers, m):
+def ncu_traffic(shape_name, layers, m):
     """DRAM bytes (read + write) per launch of the batch-1 stack kernel, from the
-    committed ncu summary (measured on a 6-layer stack, scaled per layer)."""
+    committed ncu summary of the Qwen3-4B-shaped stack (measured on 6 layers,
+    scaled per layer); None for any other shape or batch (not captured)."""
     p = os.path.join(ROOT, "profiles", "stack1_kernel_qwen3-4b-shaped_m1.md")
-    if m != 1 or not os.path.exists(p):
+    if m != 1 or shape_name != "qwen3-4b-shaped" or not os.path.exists(p):
         return None
     with open(p) as f:
         for ln in f:
@@ -370,8 +372,8 @@ def main():
     kern_ms_layer = sum(ph_ms)
     flops_layer = 2.0 * m * shape.weights_per_layer()
     tensor_tflops = flops_layer / (kern_ms_layer * 1e-3) / 1e12
-    # batch 1: the timed step is one launch of the persistent stack kernel (plus
-    # a 256-byte memset of its barrier word), so its duration is the step time
+    # up to 16 tokens the timed step is one launch of a persistent stack kernel
+    # (plus a 256-byte memset of its barrier word), so its duration is the step time
     stack_bytes = bytes_step_layer * shape.layers
     achieved = stack_bytes / (ms * 1e-3) / 1e9
     tokens = m * world * args.steps
@@ -422,10 +424,14 @@ def main():
         "compressed_weight_gbs": bytes_token * value / world / 1e9,
         "hbm_frac_of_measured": bytes_token * value / world / 1e9 / hbm,
         "roofline": ({"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                      "frac": achieved / hbm, "traffic": ncu_traffic(shape.layers, m), "peak_source": peak_src,
-                      "kernel": "stack1_kernel (persistent: RHT + decode + mma.sync, every phase of every layer)",
+                      "frac": achieved / hbm, "traffic": ncu_traffic(shape.name, shape.layers, m),
+                      "peak_source": peak_src,
+                      "kernel": ("stack1_kernel (persistent: RHT + decode + mma.sync, every phase of every layer)"
+                                 if m == 1 else
+                                 "stackn_kernel (persistent: grid-split RHT + decode + mma.sync, every phase of "
+                                 "every layer)"),
                       "bytes_per_launch": stack_bytes,
-                      "eager_phase_ms": ph_ms, "phase_bytes": pb} if m == 1 else
+                      "eager_phase_ms": ph_ms, "phase_bytes": pb} if m <= PERSISTENT_MAX_M else
                      {"bound": "hbm", "achieved": bytes_step_layer / (kern_ms_layer * 1e-3) / 1e9, "peak": hbm,
                       "unit": "GB/s", "frac": bytes_step_layer / (kern_ms_layer * 1e-3) / 1e9 / hbm,
                       "traffic": None, "peak_source": peak_src,
@@ -440,7 +446,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": "tok/s", "h2d_bytes_per_step": int(h_host.numel() * 2),
                 "d2h_bytes_per_step": int(o_host.numel() * 2)},
-        "gpu_launches": args.steps * (1 if m == 1 else 4 * shape.layers * 2),
+        "gpu_launches": args.steps * (1 if m <= PERSISTENT_MAX_M else 4 * shape.layers * 2),
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
