@@ -342,20 +342,14 @@ __device__ __forceinline__ void rht_block(RhtIn r, int blk, const DmmaParams* q,
 }
 
 // This warp's share of the phase's activations x' = RHT(x): blocks warp,
-// warp + 16, ...; the loads of up to three blocks are in flight together.
-// No CTA-wide synchronisation: each block is flagged when it is stored.
+// warp + 16, ... one after the other (holding several blocks' loads at once
+// costs register spills in the unit loops).  No CTA-wide synchronisation:
+// each block is flagged when it is stored.
 __device__ __forceinline__ void stack_rht(const DmmaParams& p, const DmmaParams* q, const float* gq,
                                           const uint32_t* signs, uint8_t* xs, volatile int* xflag, int tag,
                                           int warp) {
   const int nb = p.k / 512;
-  RhtIn in[3];
-#pragma unroll
-  for (int r = 0; r < 3; ++r)
-    if (warp + DMMA_WARPS * r < nb) in[r] = rht_table_load(p.x_bf16, warp + DMMA_WARPS * r, signs);
-#pragma unroll
-  for (int r = 0; r < 3; ++r)
-    if (warp + DMMA_WARPS * r < nb) rht_block(in[r], warp + DMMA_WARPS * r, q, gq, xs, xflag, tag);
-  for (int blk = warp + 3 * DMMA_WARPS; blk < nb; blk += DMMA_WARPS)  // k > 24576 only
+  for (int blk = warp; blk < nb; blk += DMMA_WARPS)
     rht_block(rht_table_load(p.x_bf16, blk, signs), blk, q, gq, xs, xflag, tag);
 }
 
