@@ -407,7 +407,29 @@ __device__ __forceinline__ void wait_xflag(const volatile int* xflag, int blk, i
 // XCG: the small-batch activations were written earlier in the same launch
 // (persistent stack), so they are read through L2 (ld.global.cg) instead of
 // the read-only path.
-template <int LV, int NT, bool HILO, bool XCG = false>
+// A warp's partial of one tile into its shared-memory slot (16 rows x MC
+// tokens, the layout of the global partials).
+template <int NT, bool HILO>
+__device__ __forceinline__ void dmma_slot_store(float* wslots, int slot, int g, int q, const float (&acc)[NT][4]) {
+  constexpr int MC = HILO ? 1 : NT * 8;
+  float* s = wslots + slot * 16 * MC;
+  if (HILO) {
+    if (q == 0) {
+      s[g] = acc[0][0] + acc[0][1];
+      s[g + 8] = acc[0][2] + acc[0][3];
+    }
+  } else {
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[partial_index<NT, HILO>(g, q, jt, i)] = acc[jt][i];
+  }
+}
+
+// SLOTS: tiles shared with other warps go to the warp's shared-memory slots
+// (wslots, persistent stack kernels) as soon as they end, holding no register
+// copy of the first tile until the end of the range.
+template <int LV, int NT, bool HILO, bool XCG = false, bool SLOTS = false>
 __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* smem, const uint8_t* xs, int64_t W,
                                            DmmaCursor& c, int lane, float* wslots = nullptr,
                                            const volatile int* xflag = nullptr, int xtag = 0,
@@ -518,7 +540,9 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
       } else if (iu + 1 < nunits) {
         // the range's first tile, shared with earlier warps: publish it at the
         // end (8 column tiles keep no second register copy: publish now)
-        if (NT <= 4) {
+        if (SLOTS) {
+          dmma_slot_store<NT, HILO>(wslots, 0, g, q, acc);
+        } else if (NT <= 4) {
           has_head = true;
           head_t = t;
 #pragma unroll
@@ -547,28 +571,8 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
   if (has_head || has_tail) {
     // slot 0 holds the range's first tile, slot 1 a later one
     const int tail_slot = (tail_t == (int)(c.wb / p.blocks)) ? 0 : 1;
-    if (wslots) {
-      if (HILO) {
-        if (q == 0) {
-          if (has_head) {
-            wslots[g] = hacc[0][0] + hacc[0][1];
-            wslots[g + 8] = hacc[0][2] + hacc[0][3];
-          }
-          if (has_tail) {
-            wslots[tail_slot * 16 + g] = acc[0][0] + acc[0][1];
-            wslots[tail_slot * 16 + g + 8] = acc[0][2] + acc[0][3];
-          }
-        }
-      } else {  // slot layout [16 rows][NT * 8 tokens], as the global partials
-        constexpr int MC = NT * 8;
-#pragma unroll
-        for (int jt = 0; jt < NT; ++jt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            if (has_head) wslots[partial_index<NT, HILO>(g, q, jt, i)] = hacc[jt][i];
-            if (has_tail) wslots[tail_slot * 16 * MC + partial_index<NT, HILO>(g, q, jt, i)] = acc[jt][i];
-          }
-      }
+    if (SLOTS) {
+      if (has_tail) dmma_slot_store<NT, HILO>(wslots, tail_slot, g, q, acc);  // the head is already in slot 0
     } else {
       dmma_publish<NT, HILO>(p, W, g, q, has_head, head_t, hacc, has_tail, tail_t, tail_slot, acc);
     }

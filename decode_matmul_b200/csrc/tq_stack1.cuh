@@ -460,7 +460,8 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
               xflag, f, warp);
     if (fetch) slots[((f + 2) & 3) * PARAM_QUADS + tid] = nq;  // slot of phase f-2: no reader left
     if (f + 1 < nphases) stack_warp_tables(slot(f + 1), wbeg(f + 1), wfirst(f + 1), tid);  // read after the barrier
-    dmma_units<LV, 1, true>(p, smem, xs, W, c, lane, wslots + warp * 32, xflag, f, sp.status, sp.spin_limit);
+    dmma_units<LV, 1, true, false, true>(p, smem, xs, W, c, lane, wslots + warp * 32, xflag, f, sp.status,
+                                           sp.spin_limit);
     // the first warp done writes the outputs of the previous phase's
     // straddling tile that starts in this CTA (its partials stay until phase
     // f+2 overwrites them), off the critical path of the slowest warp

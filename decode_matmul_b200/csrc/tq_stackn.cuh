@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stackn_kernel(const __grid_co
     grid_arrive(sp);  // x' of every token is in
     ++epoch;
     if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;
-    dmma_units<LV, NT, false, true>(p, smem, nullptr, W, c, lane, wslots + warp * 2 * SLOT);
+    dmma_units<LV, NT, false, true, true>(p, smem, nullptr, W, c, lane, wslots + warp * 2 * SLOT);
     __syncthreads();
     stackn_cta_reduce<NT>(p, wbeg(f), wfirst(f), wslots, parts(f), warp, lane);
     grid_arrive(sp);  // its __syncthreads ends every use of the warp tables, slots and slots' partials
