@@ -78,10 +78,14 @@ __host__ __device__ __forceinline__ int64_t dmma_warp_of(int64_t u, int64_t unit
   return ((u + 1) * active + units - 1) / units - 1;
 }
 
-// Shared-memory offset of the hi (n=0) or lo (n=1) fp16 quad of group G,
-// arranged so that the 8 lanes reading one MMA step hit 64 contiguous bytes.
+// Shared-memory offset of the hi (n=0) or lo (n=1) fp16 quad of group G
+// (group 16q + j of a 256-block is read by lanes with q = lane % 4 at MMA step
+// j), stored as [block][j / 2][q][n][j % 2]: a lane's quads of steps j and
+// j + 1 are one 16-byte load, and the 8 lanes that read a step pair hit 128
+// contiguous bytes.
 __device__ __forceinline__ uint32_t xs_offset(int G, int n) {
-  return (uint32_t)((((((G >> 6) << 4) + (G & 15)) << 2) + ((G >> 4) & 3)) * 16 + n * 8);
+  const int b = G >> 6, j = G & 15, q = (G >> 4) & 3;
+  return (uint32_t)((((((b << 3) + (j >> 1)) << 2) + q) * 2 + n) * 2 + (j & 1)) * 8;
 }
 
 __device__ __forceinline__ void store_hilo(uint8_t* xs, int G, float a, float b, float c, float d) {
@@ -365,14 +369,14 @@ __device__ __forceinline__ void dmma_begin(const DmmaParams& p, int64_t W, int g
   }
 }
 
-// Batch-1 activation quad of one MMA step for lanes 0-7 (lanes g = 0 / 1 hold
-// the hi / lo column); the other lanes own MMA columns that are never read
-// and skip the load (predicated, no branch).
-__device__ __forceinline__ uint2 lds_b_hilo(const uint8_t* addr, int lane) {
-  uint2 v = make_uint2(0u, 0u);
+// Batch-1 activation quads of two MMA steps for lanes 0-7 (lanes g = 0 / 1
+// hold the hi / lo column); the other lanes own MMA columns that are never
+// read and skip the load (predicated, no branch).
+__device__ __forceinline__ uint4 lds_b_hilo(const uint8_t* addr, int lane) {
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
   asm volatile(
-      "{\n .reg .pred p;\n setp.lt.u32 p, %2, 8;\n @p ld.shared.v2.u32 {%0,%1}, [%3];\n}\n"
-      : "+r"(v.x), "+r"(v.y)
+      "{\n .reg .pred p;\n setp.lt.u32 p, %4, 8;\n @p ld.shared.v4.u32 {%0,%1,%2,%3}, [%5];\n}\n"
+      : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w)
       : "r"(lane), "r"(smem_u32(addr)));
   return v;
 }
@@ -475,7 +479,8 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
       ready_rb = b >> 1;
       wait_xflag(xflag, ready_rb, xtag, status, spin_limit);
     }
-    const uint8_t* xs_lane = xs + (((b << 4) << 2) + q) * 16 + (g & 1) * 8;
+    const uint8_t* xs_lane = xs + ((((b << 3) << 2) + q) * 2 + (g & 1)) * 16;  // step pair 0
+    uint4 bw2 = make_uint4(0u, 0u, 0u, 0u);
     const uint16_t* xg_lane[NT];
     uint4 bpair[NT];
 #pragma unroll
@@ -510,8 +515,8 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
         // B columns other than the live ones (hi/lo at batch 1, tokens < m
         // otherwise) only feed C columns that are never read.
         if (HILO) {
-          const uint2 bw = lds_b_hilo(xs_lane + j * 64, lane);
-          mma_16816((j & 1) ? acc2[0] : acc[0], a, bw.x, bw.y);
+          if ((j & 1) == 0) bw2 = lds_b_hilo(xs_lane + (j >> 1) * 128, lane);  // steps j, j + 1
+          mma_16816((j & 1) ? acc2[0] : acc[0], a, (j & 1) ? bw2.z : bw2.x, (j & 1) ? bw2.w : bw2.y);
         } else {
           // one 16-byte load holds this lane's quads of steps j and j + 1
           if ((j & 1) == 0) {
