@@ -61,6 +61,7 @@ int check_weight(const tq_weight_t* w) {
   if (w->n < 1 || !k_ok(w->k)) return TQ_ERR_SHAPE;
   if (!w->codes_d || !w->scales_d || !w->codebook_d) return TQ_ERR_NULL;
   if (!aligned16(w->codes_d) || !aligned16(w->codebook_d)) return TQ_ERR_ALIGN;
+  if (reinterpret_cast<uintptr_t>(w->scales_d) & 3) return TQ_ERR_ALIGN;  // read two blocks' scales at a time
   return TQ_OK;
 }
 

@@ -137,12 +137,21 @@ __device__ __forceinline__ DmmaRows dmma_rows(const DmmaParams& p, int t, int g,
   return r;
 }
 
-__device__ __forceinline__ DmmaChunk dmma_fetch(const DmmaRows& r, int b) {
+// Codes of block b, and its scales from the scale-pair words (spa, spb) of
+// blocks (b & ~1, b | 1): loaded here when b is even or `fresh` (the first
+// block of a range), else left from the fetch of block b - 1.  Rows hold an
+// even number of blocks (k is a multiple of 512), so the words are aligned.
+__device__ __forceinline__ DmmaChunk dmma_fetch(const DmmaRows& r, int b, uint32_t& spa, uint32_t& spb,
+                                               bool fresh) {
   DmmaChunk ch;
   ch.ca = ldg_stream_u4(r.ca + b * 64);
   ch.cb = ldg_stream_u4(r.cb + b * 64);
-  ch.sa = ldg_u16(r.sa + b);
-  ch.sb = ldg_u16(r.sb + b);
+  if (fresh || (b & 1) == 0) {
+    spa = __ldg(reinterpret_cast<const uint32_t*>(r.sa + (b & ~1)));
+    spb = __ldg(reinterpret_cast<const uint32_t*>(r.sb + (b & ~1)));
+  }
+  ch.sa = (b & 1) ? (spa >> 16) : (spa & 0xFFFFu);
+  ch.sb = (b & 1) ? (spb >> 16) : (spb & 0xFFFFu);
   return ch;
 }
 
@@ -354,6 +363,7 @@ struct DmmaCursor {
   int t, b;
   DmmaRows rows;
   DmmaChunk cur;
+  uint32_t spa, spb;  // scale-pair words of block b's pair (see dmma_fetch)
 };
 
 __device__ __forceinline__ void dmma_begin(const DmmaParams& p, int64_t W, int g, int q, DmmaCursor& c) {
@@ -365,7 +375,7 @@ __device__ __forceinline__ void dmma_begin(const DmmaParams& p, int64_t W, int g
     c.t = (int)(c.wb / p.blocks);
     c.b = (int)(c.wb - (int64_t)c.t * p.blocks);
     c.rows = dmma_rows(p, c.t, g, q);
-    c.cur = dmma_fetch(c.rows, c.b);
+    c.cur = dmma_fetch(c.rows, c.b, c.spa, c.spb, true);
   }
 }
 
@@ -445,6 +455,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
   int t = c.t, b = c.b;
   DmmaRows rows = c.rows;
   DmmaChunk cur = c.cur;
+  uint32_t spa = c.spa, spb = c.spb;
   const uint32_t vofs = (uint32_t)((lane & (V - 1)) << 3);
   // two accumulator sets (even / odd code steps) halve the MMA dependency chain
   float acc[NT][4], acc2[NT][4];
@@ -472,7 +483,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
     DmmaChunk nxt;
     if (iu + 1 < nunits) {
       if (bn == 0) nrows = dmma_rows(p, tn, g, q);
-      nxt = dmma_fetch(nrows, bn);
+      nxt = dmma_fetch(nrows, bn, spa, spb, false);
     }
 
     if (HILO && xflag && (b >> 1) != ready_rb) {

@@ -373,7 +373,7 @@ __device__ __forceinline__ void stack_begin(const DmmaParams& p, const int32_t* 
     c.t = wfirst[warp];
     c.b = (int)(c.wb - (int64_t)c.t * p.blocks);
     c.rows = dmma_rows(p, c.t, lane >> 2, lane & 3);
-    c.cur = dmma_fetch(c.rows, c.b);
+    c.cur = dmma_fetch(c.rows, c.b, c.spa, c.spb, true);
   }
 }
 

@@ -74,7 +74,8 @@ extern "C" {
 #define TQ_F16 1
 
 /* One trellis-coded weight.  All pointers are device pointers (caller-owned).
- * codes_d: uint8 [n][k/4], 16-byte aligned.  scales_d: fp16 bits [n][k/256].
+ * codes_d: uint8 [n][k/4], 16-byte aligned.  scales_d: fp16 bits [n][k/256],
+ * 4-byte aligned (the kernels read the scales of two blocks at a time).
  * codebook_d: fp16 bits [8][256][4] (16384 bytes), 16-byte aligned. */
 typedef struct tq_weight {
   const uint8_t* codes_d;
