@@ -86,6 +86,12 @@ def lib():
         L.orc_viterbi.argtypes = [f64p, i64, u16p, u16p, u8p]
         L.orc_code_cost.restype = ctypes.c_double
         L.orc_code_cost.argtypes = [f64p, i64, u16p, u16p, u8p]
+        f32p = ctypes.POINTER(ctypes.c_float)
+        L.orc_viterbi32.restype = ctypes.c_float
+        L.orc_viterbi32.argtypes = [f32p, ctypes.c_int, u16p, ctypes.c_uint16, u8p]
+        L.orc_refit32.restype = ctypes.c_int
+        L.orc_refit32.argtypes = [f32p, u8p, u16p, u16p]
+        L.orc_encode32.argtypes = [f32p, i64, i64, u16p, ctypes.c_float, ctypes.c_int, u8p, u16p, f32p]
         _lib = L
     return _lib
 
@@ -217,6 +223,42 @@ def code_cost(w, k: int, codebook, scales, codes) -> float:
                                   _c(codes, np.uint8))
     return float(lib().orc_code_cost(_p(w, ctypes.c_double), k, _p(codebook, ctypes.c_uint16),
                                      _p(scales, ctypes.c_uint16), _p(codes, ctypes.c_uint8)))
+
+
+# ---- encoder with binary32 decisions -------------------------------------------
+
+def viterbi32(w, groups: int, codebook, scale_bits: int):
+    """(codes uint8 [groups], least path cost) of the binary32 Viterbi over
+    `groups` groups of w (fp32) at one fp16 scale."""
+    w, codebook = _c(w, np.float32), _c(codebook, np.uint16)
+    codes = np.zeros(groups, dtype=np.uint8)
+    j = lib().orc_viterbi32(_p(w, ctypes.c_float), groups, _p(codebook, ctypes.c_uint16), int(scale_bits),
+                            _p(codes, ctypes.c_uint8))
+    return codes, float(j)
+
+
+def refit32(w, codes, codebook):
+    """Least-squares fp16 scale bits of one 256-weight block for fixed codes,
+    or None when there is none."""
+    w, codes, codebook = _c(w, np.float32), _c(codes, np.uint8), _c(codebook, np.uint16)
+    out = np.zeros(1, dtype=np.uint16)
+    ok = lib().orc_refit32(_p(w, ctypes.c_float), _p(codes, ctypes.c_uint8), _p(codebook, ctypes.c_uint16),
+                           _p(out, ctypes.c_uint16))
+    return int(out[0]) if ok else None
+
+
+def encode32(w, codebook, gain: float, refits: int):
+    """Encode rotated weights w fp32 [n][k] (k % 256 == 0): (codes uint8
+    [n][k/4], scales fp16 bits [n][k/256], err fp32 [n][k/256])."""
+    w = _c(w, np.float32)
+    n, k = w.shape
+    codebook = _c(codebook, np.uint16)
+    codes = np.zeros((n, k // 4), dtype=np.uint8)
+    scales = np.zeros((n, k // 256), dtype=np.uint16)
+    err = np.zeros((n, k // 256), dtype=np.float32)
+    lib().orc_encode32(_p(w, ctypes.c_float), n, k, _p(codebook, ctypes.c_uint16), float(gain), int(refits),
+                       _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint16), _p(err, ctypes.c_float))
+    return codes, scales, err
 
 
 # ---- layer stack (composition of the functions above) ------------------------

@@ -37,6 +37,13 @@
  *                             scipy.linalg.hadamard (library)
  *   orc_matmul                numpy matmul (library), linearity
  *   orc_viterbi               brute force over all code sequences (tiny rows)
+ *   orc_viterbi32             brute force in binary64 (its path is optimal to
+ *                             within binary32 rounding), the binary64 Viterbi
+ *   orc_refit32               exact least-squares cases (w = 2^e * path)
+ *   orc_encode32              closed-form scales, zero-error round trips,
+ *                             monotone refits, Gaussian MSE between the
+ *                             rate-distortion bound and the best 2-bit
+ *                             scalar quantizer
  * Compile: gcc -O2 -ffp-contract=off -fPIC -shared (no fast-math).
  */
 #include <math.h>
@@ -316,4 +323,160 @@ double orc_code_cost(const double* w, int64_t k, const uint16_t* cb, const uint1
     }
   }
   return total;
+}
+
+/* ======================================================================== */
+/* Trellis encoder with binary32 decisions.                                  */
+/*                                                                           */
+/* "Pingala-8" landing page, "How it works": the groups of four weights are  */
+/* coded in order, the state carried from one group selects the values the   */
+/* next group may use, and the result lands closer to the weights at the     */
+/* same bits; a random Hadamard rotation is applied to the weights first.    */
+/* The pages give no encoding procedure.  Readings adopted here:             */
+/*  - per 256-weight block the code path of least squared error is found by  */
+/*    dynamic programming over the 8 states (Viterbi), start state 0, end    */
+/*    state free;                                                            */
+/*  - the block's fp16 scale starts at RMS(block) * gain and is refitted by  */
+/*    least squares on the chosen path (sum w*e / sum e*e, e the unscaled    */
+/*    codebook values) up to `refits` times, a refit kept only when its      */
+/*    path costs less;                                                       */
+/*  - every decision (scale roundings, path choices) is taken in binary32 in */
+/*    the order written below, so that any implementation with this order    */
+/*    chooses identical codes.  orc_viterbi above is the binary64 reference. */
+/*                                                                           */
+/* Candidate cost of code c from state s for group weights w (u = -2 w):     */
+/*   t = J[s] + N[s][c];  t = fma(u3, D3, t); ... t = fma(u0, D0, t)          */
+/* with D = fp16_RNE(scale * cb[s][c]) and N = ((D0*D0 + D1*D1) + D2*D2) +   */
+/* D3*D3 (each "a*a + r" one fma).  t equals the squared error minus |w|^2,  */
+/* a constant of the group.  The new state c & 7 keeps the least t; ties go  */
+/* to the smaller code, then the smaller predecessor state.  Sums over a     */
+/* block use the fold order: v[i] += v[i + h] for h = 128, 64, ..., 1.       */
+/* ======================================================================== */
+
+static float f32_of_f16(uint16_t h) { return (float)orc_f16_to_f64(h); }
+static uint16_t f16_of_f32(float x) { return orc_f16_from_f64((double)x); }
+
+/* Fold-order sum of n (a power of two) values; v is overwritten. */
+static float fold_sum(float* v, int n) {
+  for (int h = n / 2; h >= 1; h /= 2)
+    for (int i = 0; i < h; ++i) v[i] = v[i] + v[i + h];
+  return v[0];
+}
+
+/* Viterbi over `groups` groups (1..64) of w at fp16 scale bits `scale`.
+ * codes out: uint8 [groups].  Returns the least final path cost t (squared
+ * error minus the sum of |w_g|^2). */
+float orc_viterbi32(const float* w, int groups, const uint16_t* cb, uint16_t scale, uint8_t* codes) {
+  float D[8][256][4], N[8][256];
+  uint8_t bp[64][8];
+  float sigma = f32_of_f16(scale);
+  for (int s = 0; s < 8; ++s)
+    for (int c = 0; c < 256; ++c) {
+      for (int j = 0; j < 4; ++j) D[s][c][j] = f32_of_f16(f16_of_f32(sigma * f32_of_f16(cb[(s * 256 + c) * 4 + j])));
+      float nn = D[s][c][0] * D[s][c][0];
+      nn = fmaf(D[s][c][1], D[s][c][1], nn);
+      nn = fmaf(D[s][c][2], D[s][c][2], nn);
+      N[s][c] = fmaf(D[s][c][3], D[s][c][3], nn);
+    }
+  float J[8];
+  for (int s = 0; s < 8; ++s) J[s] = (s == 0) ? 0.0f : INFINITY;
+  for (int g = 0; g < groups; ++g) {
+    float u[4];
+    for (int j = 0; j < 4; ++j) u[j] = -2.0f * w[4 * g + j];
+    float Jn[8];
+    for (int ns = 0; ns < 8; ++ns) {
+      float best = 0.0f;
+      int bc = -1, bs = -1;
+      for (int c = ns; c < 256; c += 8)
+        for (int s = 0; s < 8; ++s) {
+          float t = J[s] + N[s][c];
+          t = fmaf(u[3], D[s][c][3], t);
+          t = fmaf(u[2], D[s][c][2], t);
+          t = fmaf(u[1], D[s][c][1], t);
+          t = fmaf(u[0], D[s][c][0], t);
+          if (bc < 0 || t < best) {
+            best = t;
+            bc = c;
+            bs = s;
+          }
+        }
+      Jn[ns] = best;
+      bp[g][ns] = (uint8_t)((bc & 0xF8) | bs);
+    }
+    memcpy(J, Jn, sizeof J);
+  }
+  int st = 0;
+  for (int s = 1; s < 8; ++s)
+    if (J[s] < J[st]) st = s;
+  float jmin = J[st];
+  for (int g = groups - 1; g >= 0; --g) {
+    codes[g] = (uint8_t)((bp[g][st] & 0xF8) | st);
+    st = bp[g][st] & 7;
+  }
+  return jmin;
+}
+
+/* Least-squares scale of one 256-weight block for fixed codes:
+ * fp16_RNE(sum w*e / sum e*e), clamped to +-65504.  Returns 0 (no refit)
+ * when sum e*e is not positive or the ratio is not a number. */
+int orc_refit32(const float* w, const uint8_t* codes, const uint16_t* cb, uint16_t* scale) {
+  float p[256], q[256];
+  for (int i = 0; i < 256; ++i) {
+    int g = i / 4, j = i % 4;
+    int s = (g == 0) ? 0 : (codes[g - 1] & 7);
+    float e = f32_of_f16(cb[(s * 256 + codes[g]) * 4 + j]);
+    p[i] = w[i] * e;
+    q[i] = e * e;
+  }
+  float num = fold_sum(p, 256), den = fold_sum(q, 256);
+  if (!(den > 0.0f)) return 0;
+  float r = num / den;
+  if (isnan(r)) return 0;
+  if (r > 65504.0f) r = 65504.0f;
+  if (r < -65504.0f) r = -65504.0f;
+  *scale = f16_of_f32(r);
+  return 1;
+}
+
+/* Encode n rows of k rotated weights (k a multiple of 256).
+ * w: fp32 [n][k]; cb: fp16 [8][256][4]; codes out uint8 [n][k/4]; scales out
+ * fp16 [n][k/256]; err out fp32 [n][k/256] = fold-order sum of (w - w_hat)^2
+ * of the chosen encoding (may be NULL). */
+void orc_encode32(const float* w, int64_t n, int64_t k, const uint16_t* cb, float gain, int refits, uint8_t* codes,
+                  uint16_t* scales, float* err) {
+  int64_t nb = k / 256;
+  for (int64_t r = 0; r < n; ++r)
+    for (int64_t b = 0; b < nb; ++b) {
+      const float* wb = w + r * k + b * 256;
+      float v[256];
+      for (int i = 0; i < 256; ++i) v[i] = wb[i] * wb[i];
+      float ss = fold_sum(v, 256);
+      float rs = sqrtf(ss * 0.00390625f) * gain;
+      if (!(rs <= 65504.0f)) rs = 65504.0f;
+      uint16_t best_scale = f16_of_f32(rs);
+      uint8_t best[64], cand[64];
+      float best_j = orc_viterbi32(wb, 64, cb, best_scale, best);
+      for (int it = 0; it < refits; ++it) {
+        uint16_t s1;
+        if (!orc_refit32(wb, best, cb, &s1) || s1 == best_scale) break;
+        float j1 = orc_viterbi32(wb, 64, cb, s1, cand);
+        if (!(j1 < best_j)) break;
+        best_j = j1;
+        best_scale = s1;
+        memcpy(best, cand, 64);
+      }
+      memcpy(codes + r * (k / 4) + b * 64, best, 64);
+      scales[r * nb + b] = best_scale;
+      if (err) {
+        float sigma = f32_of_f16(best_scale);
+        for (int i = 0; i < 256; ++i) {
+          int g = i / 4, j = i % 4;
+          int s = (g == 0) ? 0 : (best[g - 1] & 7);
+          float wh = f32_of_f16(f16_of_f32(sigma * f32_of_f16(cb[(s * 256 + best[g]) * 4 + j])));
+          float d = wb[i] - wh;
+          v[i] = d * d;
+        }
+        err[r * nb + b] = fold_sum(v, 256);
+      }
+    }
 }

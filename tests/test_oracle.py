@@ -308,6 +308,121 @@ def test_viterbi_round_trip_on_decodable_rows():
     assert np.array_equal(oracle.decode(enc[None, :], sc, cb, 1, k)[0].view(np.float16).astype(np.float64), w)
 
 
+# ---- encoder with binary32 decisions -------------------------------------------------------
+
+def _path_values(codes, cb_bits):
+    """Unscaled codebook values along a code path of one 256-block (fp64 [256])."""
+    cbv = cb_bits.view(np.float16).astype(np.float64).reshape(8, 256, 4)
+    st = np.concatenate([[0], codes[:-1] & 7])
+    return cbv[st, codes].reshape(-1)
+
+
+@pytest.mark.parametrize("groups", [1, 2, 3])
+def test_viterbi32_path_is_optimal_within_binary32(groups):
+    # brute force over all 256^groups paths in binary64 (numpy fp16 rounding)
+    cb = tqsynth.codebook(21)
+    sc = np.float16(0.02).view(np.uint16)
+    rng = np.random.default_rng(100 + groups)
+    for _ in range(3):
+        w = (rng.standard_normal(4 * groups) * 0.02).astype(np.float32)
+        codes, j = oracle.viterbi32(w, groups, cb, sc)
+        best = _brute_min_cost(w.astype(np.float64), cb, sc, groups)
+        got = oracle.code_cost(w.astype(np.float64), 4 * groups, cb, np.array([sc], np.uint16), codes)
+        wn = float((w.astype(np.float64) ** 2).sum())
+        assert got - best <= 1e-5 * wn
+        # the returned cost is the squared error minus |w|^2
+        assert abs((j + wn) - got) <= 1e-5 * wn
+
+
+def test_viterbi32_agrees_with_binary64_viterbi_on_blocks():
+    cb = tqsynth.codebook(22)
+    rng = np.random.default_rng(5)
+    same = 0
+    for trial in range(6):
+        w = rng.standard_normal(256).astype(np.float32)
+        sc = np.float16([0.8, 1.0, 1.2][trial % 3]).view(np.uint16)
+        c32, j32 = oracle.viterbi32(w, 64, cb, sc)
+        c64, cost64 = oracle.viterbi(w.astype(np.float64), 256, cb, np.array([sc], np.uint16))
+        cost32 = oracle.code_cost(w.astype(np.float64), 256, cb, np.array([sc], np.uint16), c32)
+        assert cost32 - cost64 <= 1e-5 * float((w.astype(np.float64) ** 2).sum())
+        same += int(np.array_equal(c32, c64))
+    assert same >= 4  # identical paths except on near-ties
+
+
+def test_viterbi32_round_trip_on_decodable_block():
+    cb = tqsynth.codebook(23)
+    codes = tqsynth.codes(23, 0, 0, 1, 256)[0]
+    sc = np.float16(0.75).view(np.uint16)
+    w = oracle.decode(codes[None, :], np.array([[sc]], np.uint16), cb, 1, 256).view(np.float16)
+    w = w.astype(np.float32)[0]
+    enc, j = oracle.viterbi32(w, 64, cb, sc)
+    cost = oracle.code_cost(w.astype(np.float64), 256, cb, np.array([sc], np.uint16), enc)
+    assert cost == 0.0
+    assert abs(j + float((w.astype(np.float64) ** 2).sum())) <= 1e-4
+
+
+@pytest.mark.parametrize("lam,bits", [(0.5, 0x3800), (0.125, 0x3000), (-0.25, 0xB400), (2.0, 0x4000)])
+def test_refit32_exact_for_power_of_two_multiples(lam, bits):
+    # w = lam * e with lam a power of two: sum w*e = lam * sum e*e exactly
+    cb = tqsynth.codebook(24)
+    codes = tqsynth.codes(24, 0, 0, 1, 256)[0]
+    w = (lam * _path_values(codes, cb)).astype(np.float32)
+    assert oracle.refit32(w, codes, cb) == bits
+
+
+def test_refit32_none_without_energy():
+    cb = np.zeros(8 * 256 * 4, dtype=np.uint16)  # all-zero codebook
+    w = np.ones(256, dtype=np.float32)
+    assert oracle.refit32(w, np.zeros(64, np.uint8), cb) is None
+
+
+@pytest.mark.parametrize("gain,bits", [(0.5, 0x3E00), (0.25, 0x3A00)])
+def test_encode32_initial_scale_closed_form(gain, bits):
+    # |w| = 3 everywhere: RMS = 3 exactly, scale = fp16(3 * gain)
+    rng = np.random.default_rng(3)
+    w = (3.0 * rng.choice([-1.0, 1.0], size=(2, 512))).astype(np.float32)
+    _, scales, _ = oracle.encode32(w, tqsynth.codebook(25), gain, 0)
+    assert (scales == bits).all()
+
+
+def test_encode32_zero_block():
+    w = np.zeros((1, 512), dtype=np.float32)
+    codes, scales, err = oracle.encode32(w, tqsynth.codebook(26), 1.0, 2)
+    assert (codes == 0).all() and (scales == 0).all() and (err == 0).all()
+
+
+def test_encode32_err_is_decoded_squared_error():
+    cb = tqsynth.codebook(27)
+    w = np.random.default_rng(8).standard_normal((3, 768)).astype(np.float32)
+    codes, scales, err = oracle.encode32(w, cb, 1.0, 1)
+    wh = oracle.decode(codes, scales, cb, 3, 768).view(np.float16).astype(np.float64)
+    want = ((w.astype(np.float64) - wh) ** 2).reshape(3, 3, 256).sum(axis=2)
+    assert np.allclose(err, want, rtol=1e-5, atol=0)
+
+
+def test_encode32_refits_never_increase_error():
+    cb = tqsynth.codebook(28)
+    w = np.random.default_rng(9).standard_normal((2, 1024)).astype(np.float32)
+    prev = None
+    for r in range(4):
+        _, _, err = oracle.encode32(w, cb, 1.0, r)
+        if prev is not None:
+            assert (err <= prev * (1 + 1e-6)).all()
+        prev = err
+
+
+def test_encode32_gaussian_mse_between_bounds():
+    # Unit Gaussian weights at 2.0625 bits per weight: the distortion-rate
+    # bound is 2^(-2R); the best 2-bit scalar quantizer (Lloyd-Max, 4 levels)
+    # reaches 0.1175 (Max 1960).  The trellis must land between the two.
+    cb = tqsynth.codebook(0)
+    gain = 1.0 / math.sqrt(float((cb.view(np.float16).astype(np.float64) ** 2).mean()))
+    w = np.random.default_rng(11).standard_normal((4, 1024)).astype(np.float32)
+    _, _, err = oracle.encode32(w, cb, gain, 1)
+    mse = float(err.astype(np.float64).sum()) / w.size
+    assert 2.0 ** (-2 * 2.0625) < mse < 0.1175
+
+
 # ---- stack -------------------------------------------------------------------------------
 
 def test_alpha_second_moment_closed_form():
