@@ -17,14 +17,15 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 (TQ_OK, TQ_ERR_SHAPE, TQ_ERR_ALIGN, TQ_ERR_NULL, TQ_ERR_ARCH, TQ_ERR_WORKSPACE, TQ_ERR_CUDA, TQ_ERR_TIMEOUT,
- TQ_ERR_SCRATCH) = range(9)
+ TQ_ERR_SCRATCH, TQ_ERR_VALUE) = range(10)
+TQ_ENCODE_MAX_REFITS = 16
 TQ_F32, TQ_F16 = 0, 1
 OPS = ("q", "k", "v", "o", "gate", "up", "down")
 
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
            "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
-           "tq_layer_stack_buffers", "tq_layer_stack_outputs")
+           "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode")
 
 
 class TqError(RuntimeError):
@@ -82,6 +83,7 @@ def _lib():
             "tq_layer_stack": ([LY, i32, vp, i32, u64, vp, vp, sz, vp], ctypes.c_int),
             "tq_layer_stack_buffers": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_layer_stack_outputs": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+            "tq_encode": ([vp, i32, i32, vp, ctypes.c_float, i32, vp, vp, vp, vp], ctypes.c_int),
             "tq_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "tq_last_cuda_error": ([], ctypes.c_int),
         }
@@ -271,3 +273,23 @@ class StackArgs:
 def tq_layer_stack(args: StackArgs, h_in, seed: int, h_out, ws, stream=None):
     _ok(_lib().tq_layer_stack(args.arr, args.n_layers, _ptr(h_in), args.m, seed, _ptr(h_out), _ptr(ws), ws.numel(),
                               _stream(stream)), "tq_layer_stack")
+
+
+def tq_encode(w_rot, codebook, gain: float, refits: int = 1, codes=None, scales=None, err=None, want_err=True,
+              stream=None):
+    """Trellis-encode rotated weights w_rot (fp32 [n][k] on the device).
+    codebook: int16 (fp16 bits) tensor [8*256*4] on the device.  Returns
+    (codes uint8 [n][k/4], scales int16 fp16 bits [n][k/256], err fp32
+    [n][k/256] or None)."""
+    import torch
+    n, k = w_rot.shape
+    dev = w_rot.device
+    if codes is None:
+        codes = torch.empty((n, k // 4), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((n, k // 256), dtype=torch.int16, device=dev)
+    if err is None and want_err:
+        err = torch.empty((n, k // 256), dtype=torch.float32, device=dev)
+    _ok(_lib().tq_encode(_ptr(w_rot), n, k, _ptr(codebook), float(gain), int(refits), _ptr(codes), _ptr(scales),
+                         _ptr(err), _stream(stream)), "tq_encode")
+    return codes, scales, err

@@ -3,9 +3,13 @@
     python -m decode_matmul_b200.cases gemv --n 32768 --k 16384 [--reps 10]
     python -m decode_matmul_b200.cases gemm --n 19456 --k 2560 --m 512 [--reps 10]
     python -m decode_matmul_b200.cases rht  --m 512 --k 9728 [--reps 10]
+    python -m decode_matmul_b200.cases encode --n 4096 --k 14336 [--refits 0] [--reps 5]
 
 Runs `reps` launches after 3 warm-up launches and prints the mean time per
-launch (CUDA events) with the algorithmic bytes or FLOPs per launch.  The
+launch (CUDA events) with the algorithmic bytes or FLOPs per launch.  For the
+encoder the work unit is one Viterbi candidate (a code from a predecessor
+state for one group: 5 FP32 operations); with --refits 0 every block runs
+exactly one pass of 64 groups x 2048 candidates.  The
 same command line is what the ncu summaries under profiles/ were taken on.
 """
 from __future__ import annotations
@@ -28,7 +32,8 @@ def main(argv=None):
     import tqsynth
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemv", "gemm", "rht"])
+    ap.add_argument("op", choices=["gemv", "gemm", "rht", "encode"])
+    ap.add_argument("--refits", type=int, default=0)
     ap.add_argument("--n", type=int, default=32768)
     ap.add_argument("--k", type=int, default=16384)
     ap.add_argument("--m", type=int, default=1)
@@ -36,7 +41,19 @@ def main(argv=None):
     a = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
 
-    if a.op == "rht":
+    if a.op == "encode":
+        g = torch.Generator(device=dev)
+        g.manual_seed(0)
+        w = torch.randn((a.n, a.k), device=dev, generator=g)
+        cbh = tqsynth.codebook(0)
+        cb = torch.from_numpy(cbh.reshape(-1).view(np.int16)).to(dev)
+        gain = float(np.float32(1.0 / np.sqrt((tqsynth.f16_to_f64(cbh) ** 2).mean())))
+        codes = torch.empty((a.n, a.k // 4), dtype=torch.uint8, device=dev)
+        scales = torch.empty((a.n, a.k // 256), dtype=torch.int16, device=dev)
+        err = torch.empty((a.n, a.k // 256), dtype=torch.float32, device=dev)
+        run = lambda: tq.tq_encode(w, cb, gain, a.refits, codes, scales, err)  # noqa: E731
+        work, unit = a.n * (a.k // 256) * 64.0 * 2048, "cand"
+    elif a.op == "rht":
         x = torch.from_numpy(tqsynth.activations(0, a.m, a.k).view(np.int16)).to(dev)
         out = torch.empty((a.m, a.k), dtype=torch.float16, device=dev)
         run = lambda: tq.tq_rht(x, 1, tq.TQ_F16, out=out)  # noqa: E731
@@ -69,6 +86,13 @@ def main(argv=None):
     rate = work / (ms * 1e-3)
     print(f"{a.op} n={a.n} k={a.k} m={a.m}: {ms * 1e3:.2f} us/launch, "
           f"{rate / 1e9:.1f} G{unit}/s ({work:.4g} {unit} per launch)")
+    if a.op == "encode":
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        peak = sms * 128 * 1.965e9 / 5.0  # candidates/s at 5 FP32 operations each, 1965 MHz
+        mse = float(err.double().sum().item()) / (a.n * a.k)
+        print(f"  {a.n * a.k / (ms * 1e-3) / 1e9:.2f} G weights/s; candidate rate {rate / peak:.3f} of the "
+              f"FP32 bound ({peak / 1e12:.2f} T cand/s); refits={a.refits}; MSE/var {mse:.5f} "
+              f"(best 2-bit scalar quantizer 0.1175, distortion-rate bound {2 ** (-2 * 2.0625):.4f})")
 
 
 if __name__ == "__main__":

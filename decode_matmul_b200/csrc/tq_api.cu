@@ -8,6 +8,7 @@
 #include "tq_common.cuh"
 #include "tq_decode.cuh"
 #include "tq_dmma.cuh"
+#include "tq_encode.cuh"
 #include "tq_rht.cuh"
 #include "tq_stack1.cuh"
 #include "tq_stackn.cuh"
@@ -919,6 +920,29 @@ int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void
   return dmma_run(p, true, ws, TQ_GEMV_NOALLOC_SCRATCH_BYTES, sms, s);
 }
 
+int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
+              uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream) {
+  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
+  if (!(gain > 0.0f) || !(gain <= 3.0e38f) || refits < 0 || refits > TQ_ENCODE_MAX_REFITS) return TQ_ERR_VALUE;
+  if (!w_rot_d || !codebook_d || !codes_d || !scales_d) return TQ_ERR_NULL;
+  if (!aligned16(w_rot_d) || !aligned16(codebook_d) || !aligned16(codes_d)) return TQ_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(scales_d) & 3) || (reinterpret_cast<uintptr_t>(err_d) & 3)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  int st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int b = 0;
+    TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, tq::encode_kernel, tq::kEncThreads, 0));
+    per_sm = b > 0 ? b : 1;
+  }
+  const long long blocks = (long long)n * (k / 256);
+  long long grid = (long long)sms * per_sm;
+  if (grid > blocks) grid = blocks;
+  return launch(tq::encode_kernel, dim3((unsigned)grid), dim3(tq::kEncThreads), 0, (cudaStream_t)stream, w_rot_d,
+                blocks, codebook_d, gain, (int)refits, codes_d, scales_d, err_d);
+}
+
 const char* tq_status_string(int status) {
   switch (status) {
     case TQ_OK: return "ok";
@@ -930,6 +954,7 @@ const char* tq_status_string(int status) {
     case TQ_ERR_CUDA: return "CUDA runtime error (see tq_last_cuda_error)";
     case TQ_ERR_TIMEOUT: return "bounded device wait expired";
     case TQ_ERR_SCRATCH: return "problem larger than the built-in scratch of tq_gemv_noalloc (n > 262128)";
+    case TQ_ERR_VALUE: return "a scalar argument is out of range";
     default: return "unknown status";
   }
 }

@@ -68,6 +68,7 @@ extern "C" {
 #define TQ_ERR_CUDA 6      /* a CUDA runtime call failed; tq_last_cuda_error() has its code */
 #define TQ_ERR_TIMEOUT 7   /* a bounded device-side wait expired (reported by the status word) */
 #define TQ_ERR_SCRATCH 8   /* the problem does not fit the built-in scratch of tq_gemv_noalloc */
+#define TQ_ERR_VALUE 9     /* a scalar argument (not a size) is out of range */
 
 /* output element types */
 #define TQ_F32 0
@@ -237,6 +238,41 @@ TQ_API int tq_layer_stack_buffers(const tq_layer_t* layers, int32_t n_layers, in
  * pages define no such query.  TQ_ERR_NULL / TQ_ERR_SHAPE as
  * tq_layer_stack_workspace. */
 TQ_API int tq_layer_stack_outputs(const tq_layer_t* layers, int32_t n_layers, int32_t m, size_t offsets[4]);
+
+/* ---- encoder ----------------------------------------------------------------
+ * Trellis encoder ("Pingala-8" landing page, "How it works": groups of four
+ * weights are coded in order, the state carried from one group selects the
+ * values the next may use, and a random Hadamard rotation is applied to the
+ * weights before encoding).  The pages give no encoding procedure; this is
+ * the one the library implements, per row and 256-weight block b:
+ *   1. scale = fp16_RNE(min(sqrt(sum_i w_i^2 / 256) * gain, 65504));
+ *   2. the code path of least squared error sum_i (w_i - W_i)^2, W the
+ *      decoded block (the "weight" line of the format above), from state 0
+ *      with a free end state, by dynamic programming over the 8 states;
+ *   3. up to `refits` times: scale' = fp16_RNE(sum w_i e_i / sum e_i^2), e the
+ *      unscaled codebook values on the path (clamped to +-65504); a new path
+ *      at scale'; kept only when it costs less, otherwise stop (also when
+ *      scale' equals the scale or sum e_i^2 is not positive).
+ * Decisions are taken in binary32 in one fixed order (see tq_encode.cuh), so
+ * results are reproducible bit for bit.
+ * w_rot_d:   device fp32 [n][k], the rotated weights (tq_rht of the bf16
+ *            weight rows with TQ_F32 and the seed the activations will use),
+ *            16-byte aligned, finite; |w| should stay well inside the fp16
+ *            range (a scaled codebook entry that overflows fp16 makes that
+ *            block's result unspecified).
+ * codebook_d: fp16 bits [8][256][4], 16-byte aligned.
+ * gain:      > 0 and finite; 1 / RMS(codebook entries) matches the block RMS
+ *            to the codebook's (TQ_ERR_VALUE otherwise).
+ * refits:    0 .. TQ_ENCODE_MAX_REFITS (TQ_ERR_VALUE otherwise).
+ * codes_d:   device uint8 [n][k/4] out, 16-byte aligned.
+ * scales_d:  device fp16 bits [n][k/256] out, 4-byte aligned.
+ * err_d:     device fp32 [n][k/256] out, or NULL: per block, the squared
+ *            error of the chosen encoding summed in fold order
+ *            (v[i] += v[i + h], h = 128 ... 1), 4-byte aligned.
+ * k must be a positive multiple of 512 and n >= 1 (TQ_ERR_SHAPE). */
+#define TQ_ENCODE_MAX_REFITS 16
+TQ_API int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
+                     uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream);
 
 /* Human-readable text of a status code (static storage). */
 TQ_API const char* tq_status_string(int status);

@@ -116,5 +116,28 @@ def test_stack_phase_seed_matches_oracle():
 
 
 def test_status_strings():
-    for st in range(8):
+    for st in range(10):
         assert len(tq.lib().tq_status_string(st)) > 0
+    assert tq.lib().tq_status_string(99) == b"unknown status"
+
+
+def test_encode_argument_checks():
+    L = tq.lib()
+    f = ctypes.c_float
+    ok = dict(w=16, n=4, k=512, cb=16, gain=f(1.0), refits=1, codes=16, scales=16, err=16)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.tq_encode(a["w"], a["n"], a["k"], a["cb"], a["gain"], a["refits"], a["codes"], a["scales"],
+                           a["err"], None)
+
+    for n, k in [(0, 512), (4, 256), (4, 0), (4, 768)]:
+        assert call(n=n, k=k) == tq.TQ_ERR_SHAPE
+    for g in [0.0, -1.0, float("inf"), float("nan")]:
+        assert call(gain=f(g)) == tq.TQ_ERR_VALUE
+    assert call(refits=-1) == tq.TQ_ERR_VALUE
+    assert call(refits=tq.TQ_ENCODE_MAX_REFITS + 1) == tq.TQ_ERR_VALUE
+    for name in ("w", "cb", "codes", "scales"):
+        assert call(**{name: None}) == tq.TQ_ERR_NULL
+    for name, v in (("w", 20), ("cb", 24), ("codes", 40), ("scales", 18), ("err", 22)):
+        assert call(**{name: v}) == tq.TQ_ERR_ALIGN

@@ -17,6 +17,10 @@ stack -- and the value ranges of the format):
   scales     fp16_RNE(0.005 + 0.025*u), u = (draw >> 11) * 2^-53 (U[0.005, 0.03])
   codebook   fp16_RNE(z), z ~ N(0,1) by Box-Muller, [8][256][4]
   x          bf16_RNE(z), z ~ N(0,1) by Box-Muller, [m][k]
+  dense W    bf16_RNE(std * z * (gain if u < rate else 1)), [n][k]: unquantized
+             weight rows for the encoder (z ~ N(0,1); u a second uniform stream
+             marks outliers)
+  W rows     fp32_RNE(std * z), [n][k]: stand-in for already rotated weights
 Box-Muller for element t: u1 = ((draw(2t) >> 11) + 1) * 2^-53,
 u2 = (draw(2t+1) >> 11) * 2^-53, z = sqrt(-2 ln u1) * cos(2 pi u2).
 """
@@ -32,6 +36,7 @@ OPS = ("q", "k", "v", "o", "gate", "up", "down")
 
 TAG_CODEBOOK = 0xC0DEB00C
 TAG_ACTIVATION = 0xAC7
+TAG_DENSE = 0xDE45E000
 
 
 def mix64_int(z: int) -> int:
@@ -145,6 +150,24 @@ def activations(seed: int, m: int, k: int, stream: int = 0) -> np.ndarray:
     """bf16 bits [m][k], N(0,1).  `stream` selects an independent stream."""
     kk = key(seed, TAG_ACTIVATION ^ (stream << 12))
     return bf16_bits(_normals(kk, 0, m * k)).reshape(m, k)
+
+
+def dense_weights(seed: int, n: int, k: int, std: float = 0.02, outlier_rate: float = 0.0,
+                  outlier_gain: float = 8.0) -> np.ndarray:
+    """bf16 bits [n][k]: unquantized weight rows, N(0, std^2) with a fraction
+    `outlier_rate` of entries multiplied by `outlier_gain`."""
+    z = _normals(key(seed, TAG_DENSE), 0, n * k) * std
+    if outlier_rate > 0.0:
+        u = _unit(draws(key(seed, TAG_DENSE | 1), 0, n * k))
+        z = np.where(u < outlier_rate, z * outlier_gain, z)
+    return bf16_bits(z).reshape(n, k)
+
+
+def weight_rows_f32(seed: int, n: int, k: int, std: float = 1.0, row0: int = 0) -> np.ndarray:
+    """fp32 [n][k]: N(0, std^2) rows row0 .. row0+n-1 of one seeded matrix
+    with k columns (a stand-in for rotated weights)."""
+    z = _normals(key(seed, TAG_DENSE | 2), row0 * k, n * k) * std
+    return z.astype(np.float32).reshape(n, k)
 
 
 def pack_bytes(n: int, k: int) -> int:
