@@ -23,16 +23,17 @@
 //       predecessor state; block sums in fold order v[i] += v[i+h],
 //       h = 128, 64, ..., 1.
 //
-// Work split.  One CTA of 256 threads encodes one block at a time (grid-stride
-// over the n * k/256 blocks).  Warp w evaluates predecessor state s = w; lane
-// l serves new state ns = l & 7 and the eight codes c = 8*(8*(l>>3) + i) + ns,
-// i = 0..7, whose scaled entries and norms it keeps in registers for the whole
-// pass.  Per group: eight candidates per lane, a minimum over the four lanes
-// that share ns (two shuffles), one shared-memory exchange between the eight
-// warps with one barrier, after which warp s reduces the eight predecessors of
-// new state s and lane 0 records the back-pointer (code high bits | state).
-// The bound is the FP32 pipe: 5 FP32 operations per candidate, 2048
-// candidates per group.
+// Work split.  One CTA of 128 threads encodes one block at a time (grid-stride
+// over the n * k/256 blocks).  Warp w evaluates the predecessor states
+// s = 2w and 2w+1; lane l serves new state ns = l & 7 and the eight codes
+// c = 8*(8*(l>>3) + i) + ns, i = 0..7, whose scaled entries and norms (for both
+// of its states) it keeps in registers for the whole pass.  Per group: sixteen
+// candidates per lane, a minimum over the four lanes that share ns (two
+// shuffles), one shared-memory exchange between the four warps with one
+// barrier, after which warp w reduces the four partial minima of new states 2w
+// (lanes 0-15) and 2w+1 (lanes 16-31) and records their back-pointers (code
+// high bits | predecessor state).  The bound is the FP32 pipe: 5 FP32
+// operations per candidate, 2048 candidates per group.
 #pragma once
 
 #include <stddef.h>
@@ -41,15 +42,16 @@
 
 namespace tq {
 
-constexpr int kEncThreads = 256;
+constexpr int kEncWarps = 4;                 // each warp: two predecessor states
+constexpr int kEncThreads = 32 * kEncWarps;  // two weights of the block per thread
 
 struct EncShared {
   float w[256];          // the block's rotated weights
   uint8_t cur[64];       // codes of the last pass (16-byte aligned: offset 1024)
   uint8_t best[64];      // codes of the best pass so far (offset 1088)
-  float red[2][256];     // fold-sum scratch
-  float kt[2][8][8];     // per group: [buffer][predecessor s][new state] least cost
-  uint32_t kc[2][8][8];  //   and its code
+  float red[2][128];     // fold-sum scratch
+  float kt[2][8][4];     // per group: [buffer][new state][warp] least cost
+  uint32_t kc[2][8][4];  //   and its key (code << 3 | predecessor state)
   uint8_t bp[64][8];     // back-pointers: (code & 0xF8) | predecessor state
   float jf[8];           // final path cost per end state
   float bc[2];           // broadcast slots
@@ -60,17 +62,13 @@ __device__ __forceinline__ float enc_rnd16(float x) { return __half2float(__floa
 
 __device__ __forceinline__ uint16_t enc_f16_bits(float x) { return __half_as_ushort(__float2half_rn(x)); }
 
-// Fold-order sums of two values held one per thread (v[i] += v[i + h] for
-// h = 128 ... 1), returned to every thread.
-__device__ __forceinline__ float2 enc_fold2(EncShared& S, float a, float b) {
+// Fold-order sums (v[i] += v[i + h] for h = 128 ... 1) of two 256-element
+// vectors a and b, thread t holding elements t and t + 128 of each; returned
+// to every thread.
+__device__ __forceinline__ float2 enc_fold2(EncShared& S, float a0, float a1, float b0, float b1) {
   const int tid = threadIdx.x;
-  S.red[0][tid] = a;
-  S.red[1][tid] = b;
-  __syncthreads();
-  if (tid < 128) {
-    S.red[0][tid] = __fadd_rn(S.red[0][tid], S.red[0][tid + 128]);
-    S.red[1][tid] = __fadd_rn(S.red[1][tid], S.red[1][tid + 128]);
-  }
+  S.red[0][tid] = __fadd_rn(a0, a1);
+  S.red[1][tid] = __fadd_rn(b0, b1);
   __syncthreads();
   if (tid < 64) {
     S.red[0][tid] = __fadd_rn(S.red[0][tid], S.red[0][tid + 64]);
@@ -110,60 +108,76 @@ __device__ __forceinline__ bool enc_before(float t_o, uint32_t k_o, float t, uin
 // go to `out` (shared memory) and the least final cost is returned to every
 // thread.
 __device__ float enc_viterbi(EncShared& S, const uint16_t* __restrict__ cb, uint16_t scale_bits, uint8_t* out) {
-  const int tid = threadIdx.x, s = tid >> 5, lane = tid & 31, ns = lane & 7, hq = lane >> 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, ns = lane & 7, hq = lane >> 3;
   const float sigma = __half2float(__ushort_as_half(scale_bits));
-  float D[8][4], N[8];
+  float D[2][8][4], N[2][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t c = ((uint32_t)(hq * 8 + i) << 3) | (uint32_t)ns;
-    const uint2 e = __ldg(reinterpret_cast<const uint2*>(cb + ((((uint32_t)s << 8) | c) << 2)));
-    const float2 e01 = h2_to_f2(e.x), e23 = h2_to_f2(e.y);
-    D[i][0] = enc_rnd16(__fmul_rn(sigma, e01.x));
-    D[i][1] = enc_rnd16(__fmul_rn(sigma, e01.y));
-    D[i][2] = enc_rnd16(__fmul_rn(sigma, e23.x));
-    D[i][3] = enc_rnd16(__fmul_rn(sigma, e23.y));
-    N[i] = fmaf(D[i][3], D[i][3], fmaf(D[i][2], D[i][2], fmaf(D[i][1], D[i][1], __fmul_rn(D[i][0], D[i][0]))));
-  }
-  float J = (s == 0) ? 0.0f : __int_as_float(0x7f800000);
+  for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t s = 2 * warp + sl, c = ((uint32_t)(hq * 8 + i) << 3) | (uint32_t)ns;
+      const uint2 e = __ldg(reinterpret_cast<const uint2*>(cb + (((s << 8) | c) << 2)));
+      const float2 e01 = h2_to_f2(e.x), e23 = h2_to_f2(e.y);
+      D[sl][i][0] = enc_rnd16(__fmul_rn(sigma, e01.x));
+      D[sl][i][1] = enc_rnd16(__fmul_rn(sigma, e01.y));
+      D[sl][i][2] = enc_rnd16(__fmul_rn(sigma, e23.x));
+      D[sl][i][3] = enc_rnd16(__fmul_rn(sigma, e23.y));
+      N[sl][i] = fmaf(D[sl][i][3], D[sl][i][3],
+                      fmaf(D[sl][i][2], D[sl][i][2], fmaf(D[sl][i][1], D[sl][i][1], __fmul_rn(D[sl][i][0], D[sl][i][0]))));
+    }
+  const float inf = __int_as_float(0x7f800000);
+  float J0 = (warp == 0) ? 0.0f : inf, J1 = inf;  // path costs of states 2w and 2w+1
   for (int g = 0; g < 64; ++g) {
     const float4 wg = *reinterpret_cast<const float4*>(S.w + 4 * g);
     const float u0 = -2.0f * wg.x, u1 = -2.0f * wg.y, u2 = -2.0f * wg.z, u3 = -2.0f * wg.w;
-    float bt = 0.0f;
-    int bi = 0;
+    // candidate index x = 2i + sl orders the lane's candidates by (code, state)
+    float tv[16];
+    int ti[16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float t = __fadd_rn(J, N[i]);
-      t = fmaf(u3, D[i][3], t);
-      t = fmaf(u2, D[i][2], t);
-      t = fmaf(u1, D[i][1], t);
-      t = fmaf(u0, D[i][0], t);
-      if (i == 0 || t < bt) {
-        bt = t;
-        bi = i;
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        float t = __fadd_rn(sl ? J1 : J0, N[sl][i]);
+        t = fmaf(u3, D[sl][i][3], t);
+        t = fmaf(u2, D[sl][i][2], t);
+        t = fmaf(u1, D[sl][i][1], t);
+        tv[2 * i + sl] = fmaf(u0, D[sl][i][0], t);
+        ti[2 * i + sl] = 2 * i + sl;
       }
-    }
-    uint32_t bc = ((uint32_t)(hq * 8 + bi) << 3) | (uint32_t)ns;
+    // least (t, x) by a tree; the right operand holds the larger x, so it wins
+    // only when strictly smaller
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+      for (int x = 0; x < 16; x += 2 * h)
+        if (tv[x + h] < tv[x]) {
+          tv[x] = tv[x + h];
+          ti[x] = ti[x + h];
+        }
+    float bt = tv[0];
+    uint32_t bk = ((((uint32_t)(hq * 8 + (ti[0] >> 1)) << 3) | (uint32_t)ns) << 3) | (uint32_t)(2 * warp + (ti[0] & 1));
 #pragma unroll
     for (int o = 8; o <= 16; o <<= 1) {
       const float to = __shfl_xor_sync(0xffffffffu, bt, o);
-      const uint32_t co = __shfl_xor_sync(0xffffffffu, bc, o);
-      if (enc_before(to, co, bt, bc)) {
+      const uint32_t ko = __shfl_xor_sync(0xffffffffu, bk, o);
+      if (enc_before(to, ko, bt, bk)) {
         bt = to;
-        bc = co;
+        bk = ko;
       }
     }
     const int buf = g & 1;
     if (hq == 0) {
-      S.kt[buf][s][ns] = bt;
-      S.kc[buf][s][ns] = bc;
+      S.kt[buf][ns][warp] = bt;
+      S.kc[buf][ns][warp] = bk;
     }
     __syncthreads();
-    // warp s now owns new state s; lane & 7 is the predecessor state
-    const int sp = lane & 7;
-    float t2 = S.kt[buf][sp][s];
-    uint32_t k2 = (S.kc[buf][sp][s] << 3) | (uint32_t)sp;
+    // warp w now owns new states 2w (lanes 0-15) and 2w+1 (lanes 16-31);
+    // lane & 3 picks the partial minimum of one warp
+    const int nn = 2 * warp + (lane >> 4);
+    float t2 = S.kt[buf][nn][lane & 3];
+    uint32_t k2 = S.kc[buf][nn][lane & 3];
 #pragma unroll
-    for (int o = 1; o <= 4; o <<= 1) {
+    for (int o = 1; o <= 2; o <<= 1) {
       const float to = __shfl_xor_sync(0xffffffffu, t2, o);
       const uint32_t ko = __shfl_xor_sync(0xffffffffu, k2, o);
       if (enc_before(to, ko, t2, k2)) {
@@ -171,10 +185,14 @@ __device__ float enc_viterbi(EncShared& S, const uint16_t* __restrict__ cb, uint
         k2 = ko;
       }
     }
-    J = t2;
-    if (lane == 0) S.bp[g][s] = (uint8_t)(((k2 >> 3) & 0xF8u) | (k2 & 7u));
+    J0 = __shfl_sync(0xffffffffu, t2, 0);
+    J1 = __shfl_sync(0xffffffffu, t2, 16);
+    if ((lane & 15) == 0) S.bp[g][nn] = (uint8_t)(((k2 >> 3) & 0xF8u) | (k2 & 7u));
   }
-  if (lane == 0) S.jf[s] = J;
+  if (lane == 0) {
+    S.jf[2 * warp] = J0;
+    S.jf[2 * warp + 1] = J1;
+  }
   __syncthreads();
   if (tid == 0) {
     int st = 0;
@@ -192,22 +210,23 @@ __device__ float enc_viterbi(EncShared& S, const uint16_t* __restrict__ cb, uint
 }
 
 // Encode n rows x k rotated weights (see the file comment).  blocks = n * k/256.
-__global__ void __launch_bounds__(kEncThreads, 3)
+__global__ void __launch_bounds__(kEncThreads, 4)
     encode_kernel(const float* __restrict__ w, long long blocks, const uint16_t* __restrict__ cb, float gain,
                   int refits, uint8_t* __restrict__ codes, uint16_t* __restrict__ scales, float* __restrict__ err) {
   __shared__ __align__(16) EncShared S;
   const int tid = threadIdx.x;
   for (long long blk = blockIdx.x; blk < blocks; blk += gridDim.x) {
-    const float wv = __ldg(w + blk * 256 + tid);
-    S.w[tid] = wv;
-    const float ss = enc_fold2(S, __fmul_rn(wv, wv), 0.0f).x;
+    const float w0 = __ldg(w + blk * 256 + tid), w1 = __ldg(w + blk * 256 + tid + 128);
+    S.w[tid] = w0;
+    S.w[tid + 128] = w1;
+    const float ss = enc_fold2(S, __fmul_rn(w0, w0), __fmul_rn(w1, w1), 0.0f, 0.0f).x;
     float rs = __fmul_rn(__fsqrt_rn(__fmul_rn(ss, 0.00390625f)), gain);
     if (!(rs <= 65504.0f)) rs = 65504.0f;
     uint16_t best_scale = enc_f16_bits(rs);
     float best_j = enc_viterbi(S, cb, best_scale, S.best);
     for (int it = 0; it < refits; ++it) {
-      const float e = enc_path_value(cb, S.best, tid);
-      const float2 nd = enc_fold2(S, __fmul_rn(wv, e), __fmul_rn(e, e));
+      const float e0 = enc_path_value(cb, S.best, tid), e1 = enc_path_value(cb, S.best, tid + 128);
+      const float2 nd = enc_fold2(S, __fmul_rn(w0, e0), __fmul_rn(w1, e1), __fmul_rn(e0, e0), __fmul_rn(e1, e1));
       if (!(nd.y > 0.0f)) break;
       float r = __fdiv_rn(nd.x, nd.y);
       if (isnan(r)) break;
@@ -225,9 +244,9 @@ __global__ void __launch_bounds__(kEncThreads, 3)
     if (tid == 0) scales[blk] = best_scale;
     if (err != nullptr) {
       const float sigma = __half2float(__ushort_as_half(best_scale));
-      const float wh = enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid)));
-      const float d = __fsub_rn(wv, wh);
-      const float e2 = enc_fold2(S, __fmul_rn(d, d), 0.0f).x;
+      const float d0 = __fsub_rn(w0, enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid))));
+      const float d1 = __fsub_rn(w1, enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid + 128))));
+      const float e2 = enc_fold2(S, __fmul_rn(d0, d0), __fmul_rn(d1, d1), 0.0f, 0.0f).x;
       if (tid == 0) err[blk] = e2;
     }
     __syncthreads();
