@@ -92,6 +92,7 @@ def lib():
         L.orc_refit32.restype = ctypes.c_int
         L.orc_refit32.argtypes = [f32p, u8p, u16p, u16p]
         L.orc_encode32.argtypes = [f32p, i64, i64, u16p, ctypes.c_float, ctypes.c_int, u8p, u16p, f32p]
+        L.orc_ldlq32.argtypes = [f32p, i64, i64, f32p, u16p, ctypes.c_float, ctypes.c_int, u8p, u16p, f32p]
         _lib = L
     return _lib
 
@@ -258,6 +259,21 @@ def encode32(w, codebook, gain: float, refits: int):
     err = np.zeros((n, k // 256), dtype=np.float32)
     lib().orc_encode32(_p(w, ctypes.c_float), n, k, _p(codebook, ctypes.c_uint16), float(gain), int(refits),
                        _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint16), _p(err, ctypes.c_float))
+    return codes, scales, err
+
+
+def ldlq32(w, u, codebook, gain: float, refits: int):
+    """Block LDLQ encoding of rotated weights w fp32 [n][k] with the Hessian
+    factor u fp32 [k][k] (block strictly upper): (codes, scales, err) as
+    encode32, err = per-block squared error of the adjusted blocks."""
+    w, u = _c(w, np.float32), _c(u, np.float32)
+    n, k = w.shape
+    codebook = _c(codebook, np.uint16)
+    codes = np.zeros((n, k // 4), dtype=np.uint8)
+    scales = np.zeros((n, k // 256), dtype=np.uint16)
+    err = np.zeros((n, k // 256), dtype=np.float32)
+    lib().orc_ldlq32(_p(w, ctypes.c_float), n, k, _p(u, ctypes.c_float), _p(codebook, ctypes.c_uint16), float(gain),
+                     int(refits), _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_uint16), _p(err, ctypes.c_float))
     return codes, scales, err
 
 

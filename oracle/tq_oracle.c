@@ -44,6 +44,10 @@
  *                             monotone refits, Gaussian MSE between the
  *                             rate-distortion bound and the best 2-bit
  *                             scalar quantizer
+ *   orc_ldlq32                U = 0 reduces to orc_encode32; the proxy-loss
+ *                             identity tr(E H E^T) = sum of block errors for
+ *                             H = (I+U)(I+U)^T (binary64 check); lower proxy
+ *                             loss than plain encoding
  * Compile: gcc -O2 -ffp-contract=off -fPIC -shared (no fast-math).
  */
 #include <math.h>
@@ -438,6 +442,42 @@ int orc_refit32(const float* w, const uint8_t* codes, const uint16_t* cb, uint16
   return 1;
 }
 
+/* Encode one 256-weight block wb: codes64 out, *scale out, *err out (fold-
+ * order sum of (w - w_hat)^2 of the chosen encoding); wh out (may be NULL):
+ * the decoded block as binary32. */
+static void encode_block32(const float* wb, const uint16_t* cb, float gain, int refits, uint8_t* codes64,
+                           uint16_t* scale, float* err, float* wh) {
+  float v[256];
+  for (int i = 0; i < 256; ++i) v[i] = wb[i] * wb[i];
+  float ss = fold_sum(v, 256);
+  float rs = sqrtf(ss * 0.00390625f) * gain;
+  if (!(rs <= 65504.0f)) rs = 65504.0f;
+  uint16_t best_scale = f16_of_f32(rs);
+  uint8_t best[64], cand[64];
+  float best_j = orc_viterbi32(wb, 64, cb, best_scale, best);
+  for (int it = 0; it < refits; ++it) {
+    uint16_t s1;
+    if (!orc_refit32(wb, best, cb, &s1) || s1 == best_scale) break;
+    float j1 = orc_viterbi32(wb, 64, cb, s1, cand);
+    if (!(j1 < best_j)) break;
+    best_j = j1;
+    best_scale = s1;
+    memcpy(best, cand, 64);
+  }
+  memcpy(codes64, best, 64);
+  *scale = best_scale;
+  float sigma = f32_of_f16(best_scale);
+  for (int i = 0; i < 256; ++i) {
+    int g = i / 4, j = i % 4;
+    int s = (g == 0) ? 0 : (best[g - 1] & 7);
+    float d = f32_of_f16(f16_of_f32(sigma * f32_of_f16(cb[(s * 256 + best[g]) * 4 + j])));
+    if (wh) wh[i] = d;
+    float e = wb[i] - d;
+    v[i] = e * e;
+  }
+  *err = fold_sum(v, 256);
+}
+
 /* Encode n rows of k rotated weights (k a multiple of 256).
  * w: fp32 [n][k]; cb: fp16 [8][256][4]; codes out uint8 [n][k/4]; scales out
  * fp16 [n][k/256]; err out fp32 [n][k/256] = fold-order sum of (w - w_hat)^2
@@ -447,36 +487,50 @@ void orc_encode32(const float* w, int64_t n, int64_t k, const uint16_t* cb, floa
   int64_t nb = k / 256;
   for (int64_t r = 0; r < n; ++r)
     for (int64_t b = 0; b < nb; ++b) {
-      const float* wb = w + r * k + b * 256;
-      float v[256];
-      for (int i = 0; i < 256; ++i) v[i] = wb[i] * wb[i];
-      float ss = fold_sum(v, 256);
-      float rs = sqrtf(ss * 0.00390625f) * gain;
-      if (!(rs <= 65504.0f)) rs = 65504.0f;
-      uint16_t best_scale = f16_of_f32(rs);
-      uint8_t best[64], cand[64];
-      float best_j = orc_viterbi32(wb, 64, cb, best_scale, best);
-      for (int it = 0; it < refits; ++it) {
-        uint16_t s1;
-        if (!orc_refit32(wb, best, cb, &s1) || s1 == best_scale) break;
-        float j1 = orc_viterbi32(wb, 64, cb, s1, cand);
-        if (!(j1 < best_j)) break;
-        best_j = j1;
-        best_scale = s1;
-        memcpy(best, cand, 64);
-      }
-      memcpy(codes + r * (k / 4) + b * 64, best, 64);
-      scales[r * nb + b] = best_scale;
-      if (err) {
-        float sigma = f32_of_f16(best_scale);
-        for (int i = 0; i < 256; ++i) {
-          int g = i / 4, j = i % 4;
-          int s = (g == 0) ? 0 : (best[g - 1] & 7);
-          float wh = f32_of_f16(f16_of_f32(sigma * f32_of_f16(cb[(s * 256 + best[g]) * 4 + j])));
-          float d = wb[i] - wh;
-          v[i] = d * d;
-        }
-        err[r * nb + b] = fold_sum(v, 256);
-      }
+      float e;
+      encode_block32(w + r * k + b * 256, cb, gain, refits, codes + r * (k / 4) + b * 64, &scales[r * nb + b], &e,
+                     NULL);
+      if (err) err[r * nb + b] = e;
     }
+}
+
+/* ======================================================================== */
+/* Block LDLQ with the trellis encoder.                                      */
+/*                                                                           */
+/* "Pingala-8" landing page, "How it works": LDLQ rounding passes each       */
+/* column's error on to the columns not yet coded.  Reading adopted: with    */
+/* the proxy Hessian factored as H = (I + U) D (I + U)^T, U strictly upper   */
+/* triangular by 256-column blocks, block b of each row is encoded from       */
+/*   w~_b = w_b + (w - w_hat)_{<b} U_{<b,b}                                  */
+/* (the errors of all earlier blocks, fed forward through U), and the error  */
+/* w - w_hat of block b is kept for the blocks after it.  Then               */
+/* (w - w_hat)(I + U) = (w~ - w_hat) blockwise, so the proxy loss            */
+/* tr((w - w_hat) H (w - w_hat)^T) equals the D-weighted quantization error   */
+/* of the adjusted blocks.  binary32, fixed order: each w~ element starts at */
+/* w and adds the products delta_i * U[i][j] by fma in ascending i.          */
+/* w: fp32 [n][k]; u: fp32 [k][k] row-major (only the block strictly upper   */
+/* part is read); outputs as orc_encode32, err = per block sum of            */
+/* (w~ - w_hat)^2 in fold order.                                             */
+/* ======================================================================== */
+void orc_ldlq32(const float* w, int64_t n, int64_t k, const float* u, const uint16_t* cb, float gain, int refits,
+                uint8_t* codes, uint16_t* scales, float* err) {
+  int64_t nb = k / 256;
+  float* delta = (float*)malloc(sizeof(float) * (size_t)k);
+  float wt[256], wh[256];
+  for (int64_t r = 0; r < n; ++r) {
+    const float* wr = w + r * k;
+    for (int64_t b = 0; b < nb; ++b) {
+      for (int j = 0; j < 256; ++j) {
+        int64_t col = b * 256 + j;
+        float acc = wr[col];
+        for (int64_t i = 0; i < b * 256; ++i) acc = fmaf(delta[i], u[i * k + col], acc);
+        wt[j] = acc;
+      }
+      float e;
+      encode_block32(wt, cb, gain, refits, codes + r * (k / 4) + b * 64, &scales[r * nb + b], &e, wh);
+      if (err) err[r * nb + b] = e;
+      for (int j = 0; j < 256; ++j) delta[b * 256 + j] = wr[b * 256 + j] - wh[j];
+    }
+  }
+  free(delta);
 }

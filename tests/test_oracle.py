@@ -423,6 +423,59 @@ def test_encode32_gaussian_mse_between_bounds():
     assert 2.0 ** (-2 * 2.0625) < mse < 0.1175
 
 
+# ---- block LDLQ ------------------------------------------------------------------------------
+
+def _cb_gain(seed):
+    cb = tqsynth.codebook(seed)
+    return cb, float(np.float32(1.0 / math.sqrt(float((cb.view(np.float16).astype(np.float64) ** 2).mean()))))
+
+
+def _proxy_loss(w, codes, scales, cb, u):
+    n, k = w.shape
+    wh = oracle.decode(codes, scales, cb, n, k).view(np.float16).astype(np.float64)
+    e = w.astype(np.float64) - wh
+    return float(((e @ (np.eye(k) + u.astype(np.float64))) ** 2).sum())
+
+
+def test_ldlq_without_feedback_is_the_plain_encoder():
+    cb, g = _cb_gain(30)
+    w = tqsynth.weight_rows_f32(30, 5, 1024)
+    got = oracle.ldlq32(w, np.zeros((1024, 1024), np.float32), cb, g, 1)
+    want = oracle.encode32(w, cb, g, 1)
+    for a, b in zip(got, want):
+        assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("gamma", [0.5, 2.0])
+def test_ldlq_proxy_loss_identity(gamma):
+    # H = (I+U)(I+U)^T: tr(E H E^T) = |E (I+U)|^2 must equal the summed squared
+    # errors of the adjusted blocks (the feedback cancels the earlier errors
+    # exactly); a wrong sign, a transposed U or feeding the adjusted-block error
+    # instead of E breaks it
+    cb, g = _cb_gain(31)
+    w = tqsynth.weight_rows_f32(31, 6, 1536)
+    u = tqsynth.hessian_factor(31, 1536, gamma)
+    codes, scales, err = oracle.ldlq32(w, u, cb, g, 1)
+    loss = _proxy_loss(w, codes, scales, cb, u)
+    assert abs(loss - float(err.astype(np.float64).sum())) <= 1e-5 * loss
+
+
+def test_ldlq_lowers_the_proxy_loss():
+    cb, g = _cb_gain(32)
+    w = tqsynth.weight_rows_f32(32, 8, 1024)
+    u = tqsynth.hessian_factor(32, 1024, 0.5)
+    c1, s1, _ = oracle.ldlq32(w, u, cb, g, 1)
+    c0, s0, _ = oracle.encode32(w, cb, g, 1)
+    assert _proxy_loss(w, c1, s1, cb, u) < 0.95 * _proxy_loss(w, c0, s0, cb, u)
+
+
+def test_hessian_factor_is_block_strictly_upper():
+    u = tqsynth.hessian_factor(33, 1024)
+    bi = np.arange(1024) // 256
+    assert (u[bi[:, None] >= bi[None, :]] == 0).all()
+    assert (u[bi[:, None] < bi[None, :]] != 0).all()
+
+
 # ---- stack -------------------------------------------------------------------------------
 
 def test_alpha_second_moment_closed_form():

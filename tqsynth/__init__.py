@@ -21,6 +21,9 @@ stack -- and the value ranges of the format):
              weight rows for the encoder (z ~ N(0,1); u a second uniform stream
              marks outliers)
   W rows     fp32_RNE(std * z), [n][k]: stand-in for already rotated weights
+  Hessian    the factor U of H = (I + U)(I + U)^T, fp32 [k][k]: U[i][j] =
+             gamma * z / sqrt(256 * (j // 256)) when i // 256 < j // 256, else 0
+             (block strictly upper, each column's feedback of norm ~gamma)
 Box-Muller for element t: u1 = ((draw(2t) >> 11) + 1) * 2^-53,
 u2 = (draw(2t+1) >> 11) * 2^-53, z = sqrt(-2 ln u1) * cos(2 pi u2).
 """
@@ -168,6 +171,16 @@ def weight_rows_f32(seed: int, n: int, k: int, std: float = 1.0, row0: int = 0) 
     with k columns (a stand-in for rotated weights)."""
     z = _normals(key(seed, TAG_DENSE | 2), row0 * k, n * k) * std
     return z.astype(np.float32).reshape(n, k)
+
+
+def hessian_factor(seed: int, k: int, gamma: float = 0.5) -> np.ndarray:
+    """fp32 [k][k]: block strictly upper factor U of a synthetic proxy Hessian
+    H = (I + U)(I + U)^T (256-column blocks)."""
+    z = _normals(key(seed, TAG_DENSE | 3), 0, k * k).reshape(k, k)
+    bi = np.arange(k) // 256
+    mask = bi[:, None] < bi[None, :]
+    norm = np.sqrt(256.0 * np.maximum(bi, 1))[None, :]
+    return np.where(mask, gamma * z / norm, 0.0).astype(np.float32)
 
 
 def pack_bytes(n: int, k: int) -> int:
