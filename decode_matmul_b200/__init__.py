@@ -25,7 +25,7 @@ OPS = ("q", "k", "v", "o", "gate", "up", "down")
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
            "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
-           "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode")
+           "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode", "tq_ldlq_workspace", "tq_ldlq_encode")
 
 
 class TqError(RuntimeError):
@@ -84,6 +84,8 @@ def _lib():
             "tq_layer_stack_buffers": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_layer_stack_outputs": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_encode": ([vp, i32, i32, vp, ctypes.c_float, i32, vp, vp, vp, vp], ctypes.c_int),
+            "tq_ldlq_workspace": ([i32, i32, szp], ctypes.c_int),
+            "tq_ldlq_encode": ([vp, i32, i32, vp, vp, ctypes.c_float, i32, vp, vp, vp, vp, sz, vp], ctypes.c_int),
             "tq_status_string": ([ctypes.c_int], ctypes.c_char_p),
             "tq_last_cuda_error": ([], ctypes.c_int),
         }
@@ -292,4 +294,31 @@ def tq_encode(w_rot, codebook, gain: float, refits: int = 1, codes=None, scales=
         err = torch.empty((n, k // 256), dtype=torch.float32, device=dev)
     _ok(_lib().tq_encode(_ptr(w_rot), n, k, _ptr(codebook), float(gain), int(refits), _ptr(codes), _ptr(scales),
                          _ptr(err), _stream(stream)), "tq_encode")
+    return codes, scales, err
+
+
+def tq_ldlq_workspace(n: int, k: int) -> int:
+    b = ctypes.c_size_t()
+    _ok(_lib().tq_ldlq_workspace(n, k, ctypes.byref(b)), "tq_ldlq_workspace")
+    return b.value
+
+
+def tq_ldlq_encode(w_rot, u, codebook, gain: float, refits: int = 1, codes=None, scales=None, err=None,
+                   want_err=True, ws=None, stream=None):
+    """Block LDLQ encoding of rotated weights w_rot (fp32 [n][k], device) with
+    the Hessian factor u (fp32 [k][k], device).  Returns (codes, scales, err)
+    as tq_encode."""
+    import torch
+    n, k = w_rot.shape
+    dev = w_rot.device
+    if codes is None:
+        codes = torch.empty((n, k // 4), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty((n, k // 256), dtype=torch.int16, device=dev)
+    if err is None and want_err:
+        err = torch.empty((n, k // 256), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(tq_ldlq_workspace(n, k), dtype=torch.uint8, device=dev)
+    _ok(_lib().tq_ldlq_encode(_ptr(w_rot), n, k, _ptr(u), _ptr(codebook), float(gain), int(refits), _ptr(codes),
+                              _ptr(scales), _ptr(err), _ptr(ws), ws.numel(), _stream(stream)), "tq_ldlq_encode")
     return codes, scales, err

@@ -920,27 +920,112 @@ int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void
   return dmma_run(p, true, ws, TQ_GEMV_NOALLOC_SCRATCH_BYTES, sms, s);
 }
 
-int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
-              uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream) {
-  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
-  if (!(gain > 0.0f) || !(gain <= 3.0e38f) || refits < 0 || refits > TQ_ENCODE_MAX_REFITS) return TQ_ERR_VALUE;
-  if (!w_rot_d || !codebook_d || !codes_d || !scales_d) return TQ_ERR_NULL;
-  if (!aligned16(w_rot_d) || !aligned16(codebook_d) || !aligned16(codes_d)) return TQ_ERR_ALIGN;
-  if ((reinterpret_cast<uintptr_t>(scales_d) & 3) || (reinterpret_cast<uintptr_t>(err_d) & 3)) return TQ_ERR_ALIGN;
-  int sms = 0;
-  int st = check_arch(&sms);
-  if (st != TQ_OK) return st;
+namespace {
+
+int enc_grid(long long blocks, int sms, int* grid) {
   static int per_sm = 0;
   if (per_sm == 0) {
     int b = 0;
     TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, tq::encode_kernel, tq::kEncThreads, 0));
     per_sm = b > 0 ? b : 1;
   }
-  const long long blocks = (long long)n * (k / 256);
-  long long grid = (long long)sms * per_sm;
-  if (grid > blocks) grid = blocks;
-  return launch(tq::encode_kernel, dim3((unsigned)grid), dim3(tq::kEncThreads), 0, (cudaStream_t)stream, w_rot_d,
-                blocks, codebook_d, gain, (int)refits, codes_d, scales_d, err_d);
+  long long g = (long long)sms * per_sm;
+  *grid = (int)(g < blocks ? g : blocks);
+  return TQ_OK;
+}
+
+int enc_check(const float* w_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
+              const uint8_t* codes_d, const uint16_t* scales_d, const float* err_d) {
+  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
+  if (!(gain > 0.0f) || !(gain <= 3.0e38f) || refits < 0 || refits > TQ_ENCODE_MAX_REFITS) return TQ_ERR_VALUE;
+  if (!w_d || !codebook_d || !codes_d || !scales_d) return TQ_ERR_NULL;
+  if (!aligned16(w_d) || !aligned16(codebook_d) || !aligned16(codes_d)) return TQ_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(scales_d) & 3) || (reinterpret_cast<uintptr_t>(err_d) & 3)) return TQ_ERR_ALIGN;
+  return TQ_OK;
+}
+
+}  // namespace
+
+int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
+              uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream) {
+  int st = enc_check(w_rot_d, n, k, codebook_d, gain, refits, codes_d, scales_d, err_d);
+  if (st != TQ_OK) return st;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  tq::EncArgs a = {};
+  a.w = w_rot_d;
+  a.ldw = k;
+  a.nbl = k / 256;
+  a.blocks = (long long)n * a.nbl;
+  a.b0 = 0;
+  a.kb = k / 256;
+  a.cb = codebook_d;
+  a.gain = gain;
+  a.refits = refits;
+  a.codes = codes_d;
+  a.scales = scales_d;
+  a.err = err_d;
+  int grid = 0;
+  st = enc_grid(a.blocks, sms, &grid);
+  if (st != TQ_OK) return st;
+  return launch(tq::encode_kernel, dim3((unsigned)grid), dim3(tq::kEncThreads), 0, (cudaStream_t)stream, a);
+}
+
+int tq_ldlq_workspace(int32_t n, int32_t k, size_t* bytes) {
+  if (!bytes) return TQ_ERR_NULL;
+  if (n < 1 || !k_ok(k)) return TQ_ERR_SHAPE;
+  *bytes = (size_t)n * (size_t)(k + 256) * sizeof(float);
+  return TQ_OK;
+}
+
+int tq_ldlq_encode(const float* w_rot_d, int32_t n, int32_t k, const float* u_d, const uint16_t* codebook_d, float gain,
+                   int32_t refits, uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* workspace_d,
+                   size_t ws_bytes, void* stream) {
+  int st = enc_check(w_rot_d, n, k, codebook_d, gain, refits, codes_d, scales_d, err_d);
+  if (st != TQ_OK) return st;
+  if (!u_d) return TQ_ERR_NULL;
+  if (!aligned16(u_d)) return TQ_ERR_ALIGN;
+  size_t need = 0;
+  tq_ldlq_workspace(n, k, &need);
+  if (!workspace_d || ws_bytes < need) return TQ_ERR_WORKSPACE;
+  if (!aligned16(workspace_d)) return TQ_ERR_ALIGN;
+  int sms = 0;
+  st = check_arch(&sms);
+  if (st != TQ_OK) return st;
+  float* delta = static_cast<float*>(workspace_d);    // [n][k]
+  float* wt = delta + (size_t)n * (size_t)k;          // [n][256]
+  const int kb = k / 256;
+  int grid = 0;
+  st = enc_grid(n, sms, &grid);
+  if (st != TQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int b = 0; b < kb; ++b) {
+    if (b > 0) {
+      st = launch(tq::ldlq_feedback_kernel, dim3((unsigned)((n + tq::kFbTile - 1) / tq::kFbTile), 256 / tq::kFbTile),
+                  dim3(256), 0, s, w_rot_d, (const float*)delta, u_d, (int)n, (int)k, b, wt);
+      if (st != TQ_OK) return st;
+    }
+    tq::EncArgs a = {};
+    a.w = b > 0 ? wt : w_rot_d;
+    a.ldw = b > 0 ? 256 : k;
+    a.nbl = 1;
+    a.blocks = n;
+    a.b0 = b;
+    a.kb = kb;
+    a.cb = codebook_d;
+    a.gain = gain;
+    a.refits = refits;
+    a.codes = codes_d;
+    a.scales = scales_d;
+    a.err = err_d;
+    a.w_ref = w_rot_d;
+    a.ldr = k;
+    a.delta = (b + 1 < kb) ? delta : nullptr;
+    st = launch(tq::encode_kernel, dim3((unsigned)grid), dim3(tq::kEncThreads), 0, s, a);
+    if (st != TQ_OK) return st;
+  }
+  return TQ_OK;
 }
 
 const char* tq_status_string(int status) {

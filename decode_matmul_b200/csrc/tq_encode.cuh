@@ -209,29 +209,51 @@ __device__ float enc_viterbi(EncShared& S, const uint16_t* __restrict__ cb, uint
   return S.bc[0];
 }
 
-// Encode n rows x k rotated weights (see the file comment).  blocks = n * k/256.
-__global__ void __launch_bounds__(kEncThreads, 4)
-    encode_kernel(const float* __restrict__ w, long long blocks, const uint16_t* __restrict__ cb, float gain,
-                  int refits, uint8_t* __restrict__ codes, uint16_t* __restrict__ scales, float* __restrict__ err) {
+// One encoder launch: blocks (r, j), r < n, j < nbl, read at w + r*ldw + 256j
+// and written to output block column b0 + j of rows with kb blocks.  With
+// `delta`, the launch also stores delta = w_ref - w_hat for those columns
+// (the error the block LDLQ feeds forward).
+struct EncArgs {
+  const float* w;
+  long long ldw;
+  long long blocks;  // n * nbl
+  int nbl, b0, kb;
+  const uint16_t* cb;
+  float gain;
+  int refits;
+  uint8_t* codes;     // [n][kb * 64]
+  uint16_t* scales;   // [n][kb]
+  float* err;         // [n][kb] or null
+  const float* w_ref; // [n][ldr], with delta
+  long long ldr;
+  float* delta;       // [n][ldr] or null
+};
+
+__global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(EncArgs a) {
   __shared__ __align__(16) EncShared S;
   const int tid = threadIdx.x;
-  for (long long blk = blockIdx.x; blk < blocks; blk += gridDim.x) {
-    const float w0 = __ldg(w + blk * 256 + tid), w1 = __ldg(w + blk * 256 + tid + 128);
+  const uint16_t* __restrict__ cb = a.cb;
+  for (long long blk = blockIdx.x; blk < a.blocks; blk += gridDim.x) {
+    const long long r = blk / a.nbl;
+    const int j = (int)(blk - r * a.nbl);
+    const float* wb = a.w + r * a.ldw + 256LL * j;
+    const long long ob = r * a.kb + a.b0 + j;
+    const float w0 = __ldg(wb + tid), w1 = __ldg(wb + tid + 128);
     S.w[tid] = w0;
     S.w[tid + 128] = w1;
     const float ss = enc_fold2(S, __fmul_rn(w0, w0), __fmul_rn(w1, w1), 0.0f, 0.0f).x;
-    float rs = __fmul_rn(__fsqrt_rn(__fmul_rn(ss, 0.00390625f)), gain);
+    float rs = __fmul_rn(__fsqrt_rn(__fmul_rn(ss, 0.00390625f)), a.gain);
     if (!(rs <= 65504.0f)) rs = 65504.0f;
     uint16_t best_scale = enc_f16_bits(rs);
     float best_j = enc_viterbi(S, cb, best_scale, S.best);
-    for (int it = 0; it < refits; ++it) {
+    for (int it = 0; it < a.refits; ++it) {
       const float e0 = enc_path_value(cb, S.best, tid), e1 = enc_path_value(cb, S.best, tid + 128);
       const float2 nd = enc_fold2(S, __fmul_rn(w0, e0), __fmul_rn(w1, e1), __fmul_rn(e0, e0), __fmul_rn(e1, e1));
       if (!(nd.y > 0.0f)) break;
-      float r = __fdiv_rn(nd.x, nd.y);
-      if (isnan(r)) break;
-      r = fminf(fmaxf(r, -65504.0f), 65504.0f);
-      const uint16_t s1 = enc_f16_bits(r);
+      float q = __fdiv_rn(nd.x, nd.y);
+      if (isnan(q)) break;
+      q = fminf(fmaxf(q, -65504.0f), 65504.0f);
+      const uint16_t s1 = enc_f16_bits(q);
       if (s1 == best_scale) break;
       const float j1 = enc_viterbi(S, cb, s1, S.cur);
       if (!(j1 < best_j)) break;
@@ -240,16 +262,99 @@ __global__ void __launch_bounds__(kEncThreads, 4)
       if (tid < 16) reinterpret_cast<uint32_t*>(S.best)[tid] = reinterpret_cast<const uint32_t*>(S.cur)[tid];
       __syncthreads();
     }
-    if (tid < 4) reinterpret_cast<uint4*>(codes + blk * 64)[tid] = reinterpret_cast<const uint4*>(S.best)[tid];
-    if (tid == 0) scales[blk] = best_scale;
-    if (err != nullptr) {
+    if (tid < 4) reinterpret_cast<uint4*>(a.codes + ob * 64)[tid] = reinterpret_cast<const uint4*>(S.best)[tid];
+    if (tid == 0) a.scales[ob] = best_scale;
+    if (a.err != nullptr || a.delta != nullptr) {
       const float sigma = __half2float(__ushort_as_half(best_scale));
-      const float d0 = __fsub_rn(w0, enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid))));
-      const float d1 = __fsub_rn(w1, enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid + 128))));
-      const float e2 = enc_fold2(S, __fmul_rn(d0, d0), __fmul_rn(d1, d1), 0.0f, 0.0f).x;
-      if (tid == 0) err[blk] = e2;
+      const float h0 = enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid)));
+      const float h1 = enc_rnd16(__fmul_rn(sigma, enc_path_value(cb, S.best, tid + 128)));
+      if (a.delta != nullptr) {
+        const long long o = r * a.ldr + 256LL * (a.b0 + j);
+        a.delta[o + tid] = __fsub_rn(__ldg(a.w_ref + o + tid), h0);
+        a.delta[o + tid + 128] = __fsub_rn(__ldg(a.w_ref + o + tid + 128), h1);
+      }
+      if (a.err != nullptr) {
+        const float d0 = __fsub_rn(w0, h0), d1 = __fsub_rn(w1, h1);
+        const float e2 = enc_fold2(S, __fmul_rn(d0, d0), __fmul_rn(d1, d1), 0.0f, 0.0f).x;
+        if (tid == 0) a.err[ob] = e2;
+      }
     }
     __syncthreads();
+  }
+}
+
+// ---- block LDLQ feedback --------------------------------------------------------
+// "Pingala-8" landing page, "How it works": LDLQ rounding passes each column's
+// error on to the columns not yet coded.  With the proxy Hessian factored as
+// H = (I + U) D (I + U)^T (U strictly upper by 256-column blocks), block b of
+// each row is encoded from
+//   wt[r][j] = w[r][256b + j] + sum_{i < 256b} delta[r][i] * U[i][256b + j],
+// each element summed by fma in ascending i (binary32), delta = w - w_hat of the
+// blocks already coded.  A plain tiled SIMT GEMM: 64 x 64 outputs per CTA,
+// a 4 x 4 register tile per thread, 32-deep k tiles in shared memory; every
+// output keeps its own accumulator, so the order per output is ascending i.
+constexpr int kFbTile = 64, kFbDepth = 32;
+
+__global__ void __launch_bounds__(256) ldlq_feedback_kernel(const float* __restrict__ w, const float* __restrict__ delta,
+                                                            const float* __restrict__ u, int n, int k, int b,
+                                                            float* __restrict__ wt) {
+  __shared__ __align__(16) float As[kFbDepth][kFbTile + 4];  // delta tile, [i][row]
+  __shared__ __align__(16) float Bs[kFbDepth][kFbTile];      // U tile, [i][col]
+  const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
+  const int row0 = blockIdx.x * kFbTile, col0 = blockIdx.y * kFbTile;
+  const long long cw = 256LL * b + col0 + tc * 4;  // this thread's first column in w / U
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = row0 + tr * 4 + i;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < n) v = __ldg(reinterpret_cast<const float4*>(w + (long long)r * k + cw));
+    acc[i][0] = v.x;
+    acc[i][1] = v.y;
+    acc[i][2] = v.z;
+    acc[i][3] = v.w;
+  }
+  const int lr = tid >> 2, lk = (tid & 3) * 8;  // delta tile loads: row lr, 8 values from lk
+  const int ui = tid >> 3, uc = (tid & 7) * 8;  // U tile loads: row ui, 8 values from uc
+  const int kend = 256 * b;
+  for (int k0 = 0; k0 < kend; k0 += kFbDepth) {
+    float4 d0 = make_float4(0.f, 0.f, 0.f, 0.f), d1 = d0;
+    if (row0 + lr < n) {
+      const float* dp = delta + (long long)(row0 + lr) * k + k0 + lk;
+      d0 = __ldg(reinterpret_cast<const float4*>(dp));
+      d1 = __ldg(reinterpret_cast<const float4*>(dp + 4));
+    }
+    const float* up = u + (long long)(k0 + ui) * k + 256LL * b + col0 + uc;
+    const float4 u0 = __ldg(reinterpret_cast<const float4*>(up)), u1 = __ldg(reinterpret_cast<const float4*>(up + 4));
+    As[lk + 0][lr] = d0.x;
+    As[lk + 1][lr] = d0.y;
+    As[lk + 2][lr] = d0.z;
+    As[lk + 3][lr] = d0.w;
+    As[lk + 4][lr] = d1.x;
+    As[lk + 5][lr] = d1.y;
+    As[lk + 6][lr] = d1.z;
+    As[lk + 7][lr] = d1.w;
+    *reinterpret_cast<float4*>(&Bs[ui][uc]) = u0;
+    *reinterpret_cast<float4*>(&Bs[ui][uc + 4]) = u1;
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kFbDepth; ++kk) {
+      const float4 av = *reinterpret_cast<const float4*>(&As[kk][tr * 4]);
+      const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tc * 4]);
+      const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = row0 + tr * 4 + i;
+    if (r < n)
+      *reinterpret_cast<float4*>(wt + (long long)r * 256 + col0 + tc * 4) =
+          make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
   }
 }
 

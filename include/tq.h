@@ -274,6 +274,30 @@ TQ_API int tq_layer_stack_outputs(const tq_layer_t* layers, int32_t n_layers, in
 TQ_API int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
                      uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream);
 
+/* Block LDLQ with the trellis encoder ("Pingala-8" landing page, "How it
+ * works": LDLQ rounding passes each column's error on to the columns not yet
+ * coded).  The proxy Hessian of the layer's inputs is given by its factor:
+ * H = (I + U) D (I + U)^T with U strictly upper triangular by 256-column
+ * blocks (U[i][j] = 0 unless i/256 < j/256; D, block diagonal, is not needed).
+ * For each 256-column block b in order, every row is encoded (as tq_encode)
+ * from
+ *   w~[r][256b + j] = w[r][256b + j] + sum_{i < 256b} E[r][i] U[i][256b + j],
+ * E = w - w_hat over the blocks already coded, each element summed by fma in
+ * ascending i in binary32.  Then E (I + U) = w~ - w_hat blockwise: the proxy
+ * loss tr(E H E^T) is the D-weighted error of the adjusted blocks.
+ * w_rot_d, codebook_d, gain, refits, codes_d, scales_d: as tq_encode.
+ * u_d:      device fp32 [k][k] row-major, 16-byte aligned (only the block
+ *           strictly upper part is read).
+ * err_d:    device fp32 [n][k/256] or NULL: per block, the fold-order sum of
+ *           (w~ - w_hat)^2.
+ * workspace_d: device, >= tq_ldlq_workspace bytes, 16-byte aligned (E and
+ *           the adjusted block; no initial contents needed).
+ * Enqueues 2*(k/256) - 1 launches on `stream`. */
+TQ_API int tq_ldlq_workspace(int32_t n, int32_t k, size_t* bytes);
+TQ_API int tq_ldlq_encode(const float* w_rot_d, int32_t n, int32_t k, const float* u_d, const uint16_t* codebook_d,
+                          float gain, int32_t refits, uint8_t* codes_d, uint16_t* scales_d, float* err_d,
+                          void* workspace_d, size_t ws_bytes, void* stream);
+
 /* Human-readable text of a status code (static storage). */
 TQ_API const char* tq_status_string(int status);
 

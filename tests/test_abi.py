@@ -141,3 +141,26 @@ def test_encode_argument_checks():
         assert call(**{name: None}) == tq.TQ_ERR_NULL
     for name, v in (("w", 20), ("cb", 24), ("codes", 40), ("scales", 18), ("err", 22)):
         assert call(**{name: v}) == tq.TQ_ERR_ALIGN
+
+
+def test_ldlq_argument_checks():
+    L = tq.lib()
+    f = ctypes.c_float
+    need = tq.tq_ldlq_workspace(4, 512)
+    assert need == 4 * (512 + 256) * 4
+    ok = dict(w=16, n=4, k=512, u=16, cb=16, gain=f(1.0), refits=1, codes=16, scales=16, err=None, ws=16,
+              wsb=need)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return L.tq_ldlq_encode(a["w"], a["n"], a["k"], a["u"], a["cb"], a["gain"], a["refits"], a["codes"],
+                                a["scales"], a["err"], a["ws"], a["wsb"], None)
+
+    assert call(k=768) == tq.TQ_ERR_SHAPE
+    assert call(gain=f(-2.0)) == tq.TQ_ERR_VALUE
+    assert call(u=None) == tq.TQ_ERR_NULL
+    assert call(u=24) == tq.TQ_ERR_ALIGN
+    assert call(ws=None) == tq.TQ_ERR_WORKSPACE
+    assert call(wsb=need - 1) == tq.TQ_ERR_WORKSPACE
+    assert call(ws=20) == tq.TQ_ERR_ALIGN
+

@@ -129,3 +129,43 @@ def test_encode_full_size_sampled_rows(tq, torch_cuda):
     for r in (0, 1, 2047, 3001, 4095):
         wc, ws, we = oracle.encode32(w[r:r + 1], cb, g, 1)
         _assert_same((codes[r:r + 1], scales[r:r + 1], err[r:r + 1]), (wc, ws, we))
+
+
+# ---- block LDLQ ------------------------------------------------------------------------------
+
+def _gpu_ldlq(tq, torch, w32, u32, cb_bits, gain, refits):
+    w_d = torch.from_numpy(np.ascontiguousarray(w32, dtype=np.float32)).cuda()
+    u_d = torch.from_numpy(np.ascontiguousarray(u32, dtype=np.float32)).cuda()
+    codes, scales, err = tq.tq_ldlq_encode(w_d, u_d, to_dev_u16(cb_bits.reshape(-1)), gain, refits)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16), err.cpu().numpy()
+
+
+@pytest.mark.parametrize("n,k,gamma,refits", [(37, 1024, 0.5, 1), (70, 1536, 2.0, 0), (1, 512, 1.0, 2)])
+def test_ldlq_bit_exact(tq, torch_cuda, n, k, gamma, refits):
+    cb = tqsynth.codebook(13)
+    w = tqsynth.weight_rows_f32(14, n, k)
+    u = tqsynth.hessian_factor(15, k, gamma)
+    g = _gain(cb)
+    _assert_same(_gpu_ldlq(tq, torch_cuda, w, u, cb, g, refits), oracle.ldlq32(w, u, cb, g, refits))
+
+
+def test_ldlq_without_feedback_equals_encode(tq, torch_cuda):
+    n, k = 20, 1024
+    cb = tqsynth.codebook(16)
+    w = tqsynth.weight_rows_f32(17, n, k)
+    g = _gain(cb)
+    _assert_same(_gpu_ldlq(tq, torch_cuda, w, np.zeros((k, k), np.float32), cb, g, 1),
+                 _gpu_encode(tq, torch_cuda, w, cb, g, 1))
+
+
+def test_ldlq_full_size_sampled_rows(tq, torch_cuda):
+    n, k = 1024, 4096
+    cb = tqsynth.codebook(0)
+    g = _gain(cb)
+    w = tqsynth.weight_rows_f32(18, n, k)
+    u = tqsynth.hessian_factor(19, k, 0.5)
+    codes, scales, err = _gpu_ldlq(tq, torch_cuda, w, u, cb, g, 1)
+    for r in (0, 511, 1023):
+        _assert_same((codes[r:r + 1], scales[r:r + 1], err[r:r + 1]), oracle.ldlq32(w[r:r + 1], u, cb, g, 1))
+
