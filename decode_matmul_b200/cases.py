@@ -4,6 +4,7 @@
     python -m decode_matmul_b200.cases gemm --n 19456 --k 2560 --m 512 [--reps 10]
     python -m decode_matmul_b200.cases rht  --m 512 --k 9728 [--reps 10]
     python -m decode_matmul_b200.cases encode --n 4096 --k 14336 [--refits 0] [--reps 5]
+    python -m decode_matmul_b200.cases ldlq --n 4096 --k 4096 [--refits 0] [--reps 3]
 
 Runs `reps` launches after 3 warm-up launches and prints the mean time per
 launch (CUDA events) with the algorithmic bytes or FLOPs per launch.  For the
@@ -32,7 +33,7 @@ def main(argv=None):
     import tqsynth
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("op", choices=["gemv", "gemm", "rht", "encode"])
+    ap.add_argument("op", choices=["gemv", "gemm", "rht", "encode", "ldlq"])
     ap.add_argument("--refits", type=int, default=0)
     ap.add_argument("--n", type=int, default=32768)
     ap.add_argument("--k", type=int, default=16384)
@@ -41,7 +42,22 @@ def main(argv=None):
     a = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
 
-    if a.op == "encode":
+    if a.op == "ldlq":
+        g = torch.Generator(device=dev)
+        g.manual_seed(0)
+        w = torch.randn((a.n, a.k), device=dev, generator=g)
+        u = torch.from_numpy(tqsynth.hessian_factor(0, a.k, 0.5)).to(dev)
+        cbh = tqsynth.codebook(0)
+        cb = torch.from_numpy(cbh.reshape(-1).view(np.int16)).to(dev)
+        gain = float(np.float32(1.0 / np.sqrt((tqsynth.f16_to_f64(cbh) ** 2).mean())))
+        codes = torch.empty((a.n, a.k // 4), dtype=torch.uint8, device=dev)
+        scales = torch.empty((a.n, a.k // 256), dtype=torch.int16, device=dev)
+        err = torch.empty((a.n, a.k // 256), dtype=torch.float32, device=dev)
+        ws = torch.empty(tq.tq_ldlq_workspace(a.n, a.k), dtype=torch.uint8, device=dev)
+        run = lambda: tq.tq_ldlq_encode(w, u, cb, gain, a.refits, codes, scales, err, ws=ws)  # noqa: E731
+        kb = a.k // 256
+        work, unit = 2.0 * a.n * 256 * 256 * kb * (kb - 1) / 2, "FLOP(feedback)"
+    elif a.op == "encode":
         g = torch.Generator(device=dev)
         g.manual_seed(0)
         w = torch.randn((a.n, a.k), device=dev, generator=g)
@@ -86,6 +102,31 @@ def main(argv=None):
     rate = work / (ms * 1e-3)
     print(f"{a.op} n={a.n} k={a.k} m={a.m}: {ms * 1e3:.2f} us/launch, "
           f"{rate / 1e9:.1f} G{unit}/s ({work:.4g} {unit} per launch)")
+    if a.op == "ldlq":
+        # the same matrix without feedback, to split the time, and the proxy loss
+        # |E (I + U)|^2 of both encodings (H = (I + U)(I + U)^T)
+        c0 = torch.empty_like(codes)
+        s0 = torch.empty_like(scales)
+        e0 = torch.empty_like(err)
+        tq.tq_encode(w, cb, gain, a.refits, c0, s0, e0)
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(a.reps):
+            tq.tq_encode(w, cb, gain, a.refits, c0, s0, e0)
+        t1.record()
+        torch.cuda.synchronize()
+        ms_enc = t0.elapsed_time(t1) / a.reps
+        ud = u.double() + torch.eye(a.k, device=dev, dtype=torch.float64)
+        losses = []
+        for cc, ss in ((codes, scales), (c0, s0)):
+            wh = tq.tq_decode(tq.DeviceWeight(cc, ss, cb, a.n, a.k)).view(torch.float16).double()
+            losses.append(float(((w.double() - wh) @ ud).pow(2).sum().item()))
+        ms_fb = ms - ms_enc
+        peak = torch.cuda.get_device_properties(0).multi_processor_count * 128 * 2 * 1.965e9
+        print(f"  plain encode {ms_enc * 1e3:.1f} us; feedback + step overhead {ms_fb * 1e3:.1f} us = "
+              f"{work / (ms_fb * 1e-3) / 1e12:.2f} TFLOP/s ({work / (ms_fb * 1e-3) / peak:.3f} of the FP32 peak "
+              f"{peak / 1e12:.1f} TFLOP/s); proxy loss LDLQ / plain = {losses[0] / losses[1]:.4f}")
     if a.op == "encode":
         sms = torch.cuda.get_device_properties(0).multi_processor_count
         peak = sms * 128 * 1.965e9 / 5.0  # candidates/s at 5 FP32 operations each, 1965 MHz
