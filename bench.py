@@ -52,6 +52,25 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+# ---- replicas (N > 1) ------------------------------------------------------------------
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (every rank calls this in the same order);
+    x itself when there is no process group."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(m: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas that each ran `steps`
+    steps of m tokens, timed by the slowest rank (ms per step)."""
+    return m * world * steps / (ms_max * steps * 1e-3)
+
+
 # ---- clocks ----------------------------------------------------------------------
 
 class ClockSampler:
@@ -334,10 +353,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
-    ms_t = torch.tensor([ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
 
     # per-phase kernel durations (eager, events between launches) for the roofline
     pb = phase_bytes(shape, m)
@@ -376,8 +392,7 @@ def main():
     # (plus a 256-byte memset of its barrier word), so its duration is the step time
     stack_bytes = bytes_step_layer * shape.layers
     achieved = stack_bytes / (ms * 1e-3) / 1e9
-    tokens = m * world * args.steps
-    value = tokens / (ms_max * args.steps * 1e-3)
+    value = replica_throughput(m, world, args.steps, ms_max)
 
     # end to end through the C ABI with host buffers: pinned h_in -> device,
     # tq_layer_stack (direct call, no graph), result -> pinned host
@@ -397,10 +412,7 @@ def main():
         ee1.record(stream)
     stream.synchronize()
     e2e_ms = ee0.elapsed_time(ee1) / args.steps
-    e2e_t = torch.tensor([e2e_ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_val = m * world / (float(e2e_t.item()) * 1e-3)
+    e2e_val = replica_throughput(m, world, 1, max_over_ranks(e2e_ms, dist, dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
