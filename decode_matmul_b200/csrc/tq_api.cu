@@ -438,10 +438,7 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
   {
     // x' fp16: row-major for the TMA of the tcgen05 GEMM, fragment order for
     // the small-batch kernel
-    const int64_t tasks = (int64_t)m * (k / 512);
-    int64_t blocks = (tasks + 7) / 8;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    st = launch(use_umma ? tq::rht_kernel<1> : tq::rht_kernel<2>, dim3((unsigned)blocks), dim3(256), 0, stream, x,
+    st = launch(use_umma ? tq::rht_kernel<1> : tq::rht_kernel<2>, tq::rht_grid(m, k), dim3(256), 0, stream, x,
                 (int)m, (int)k, seed, (void*)xr);
     if (st != TQ_OK) return st;
   }
@@ -505,13 +502,10 @@ int tq_rht(const uint16_t* x_bf16_d, int32_t m, int32_t k, uint64_t seed, void* 
   int sms = 0;
   int st = check_arch(&sms);
   if (st != TQ_OK) return st;
-  const int64_t tasks = (int64_t)m * (k / 512);
-  int64_t blocks = (tasks + 7) / 8;
-  if (blocks > (int64_t)sms * 8) blocks = (int64_t)sms * 8;
   if (out_dtype == TQ_F16)
-    return launch(tq::rht_kernel<1>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+    return launch(tq::rht_kernel<1>, tq::rht_grid(m, k), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
                   (int)k, seed, x_rot_d);
-  return launch(tq::rht_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
+  return launch(tq::rht_kernel<0>, tq::rht_grid(m, k), dim3(256), 0, (cudaStream_t)stream, x_bf16_d, (int)m,
                 (int)k, seed, x_rot_d);
 }
 

@@ -78,22 +78,47 @@ __host__ __device__ __forceinline__ int frag_pos(int k) {
   return (b << 8) + ((((j >> 1) << 3) + (q << 1) + (j & 1)) << 2) + e;
 }
 
-// Standalone RHT: grid-stride over (row, block) warp tasks.  MODE 0: fp32
-// row-major; 1: fp16 row-major; 2: fp16 in fragment order (frag_pos).
+// Standalone RHT.  CTA (blk, y) transforms 512-block `blk` of rows 8y + warp
+// (grid-stride in y): the 512 diagonal signs of the block are hashed once per
+// CTA (two per thread, packed by ballot into shared memory, before the wait for
+// the preceding kernel) and shared by its eight rows.  MODE 0: fp32 row-major;
+// 1: fp16 row-major; 2: fp16 in fragment order (frag_pos).
 template <int MODE>
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x, int m, int k, uint64_t seed,
                                                   void* __restrict__ out) {
+  __shared__ uint32_t smask[16];  // bit e % 32 of word e / 32: d[512 blk + e] = -1
+  const int blk = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t e0 = (uint32_t)blk * 512u + (uint32_t)tid;
+  const uint32_t b0 = __ballot_sync(0xffffffffu, rht_sign_negative(seed, e0));
+  const uint32_t b1 = __ballot_sync(0xffffffffu, rht_sign_negative(seed, e0 + 256u));
+  if (lane == 0) {
+    smask[warp] = b0;
+    smask[8 + warp] = b1;
+  }
+  __syncthreads();
+  const uint32_t mask16 = (smask[lane >> 1] >> ((lane & 1) * 16)) & 0xFFFFu;  // elements 16 lane .. +15
   pdl_wait();
   pdl_launch_dependents();
-  const int blocks = k / 512;
-  const long long tasks = (long long)m * blocks;
-  const int lane = threadIdx.x & 31;
-  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long t = warp0; t < tasks; t += nwarps) {
-    const int row = (int)(t / blocks), blk = (int)(t % blocks);
+  for (int rg = blockIdx.y; rg * 8 < m; rg += gridDim.y) {
+    const int row = rg * 8 + warp;
+    if (row >= m) break;
+    const int base = blk * 512 + lane * 16;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)row * k + base);
+    const uint4 p0 = src[0], p1 = src[1];
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     float v[16];
-    rht512_warp(x + (size_t)row * k, blk, seed, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // D: flip the sign bit of the bf16 value where d = -1 (exact)
+      const uint32_t f = ((mask16 >> (2 * i)) & 1u) << 15 | ((mask16 >> (2 * i + 1)) & 1u) << 31;
+      const uint32_t ww = w[i] ^ f;
+      v[2 * i] = bf16_bits_to_f(ww & 0xFFFFu);
+      v[2 * i + 1] = bf16_bits_to_f(ww >> 16);
+    }
+    wht512_warp(v);
+    const float inv = 0.044194173824159216f;  // 1/sqrt(512)
+#pragma unroll
+    for (int r = 0; r < 16; ++r) v[r] *= inv;
     const size_t o = (size_t)row * k + (size_t)blk * 512 + lane * 16;
     if (MODE == 1) {
       uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + o);
@@ -114,6 +139,12 @@ __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x
       for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
   }
+}
+
+// Grid of rht_kernel for m rows of k features.
+inline dim3 rht_grid(int m, int k) {
+  const int groups = (m + 7) / 8;
+  return dim3((unsigned)(k / 512), (unsigned)(groups < 65535 ? groups : 65535));
 }
 
 // fp16 [m][k] row-major -> fragment order (one thread per group of 4).
