@@ -40,3 +40,13 @@ def test_tcgen05_gemm_split_k_large_k():
     # 20 row tiles x 1 token tile -> split k across the blocks of k = 9728
     err = _run(2560, 9728, 64, rows=[(0, 8), (1277, 1283), (2552, 2560)])
     assert err < TOL, err
+
+
+@pytest.mark.parametrize("n,k", [(19456, 2560), (14208, 1024)])
+def test_tcgen05_gemm_split_tail_wave(n, k):
+    # more tiles than SMs with a partial last wave (304 and 222 tiles of
+    # 128 rows x 256 tokens on 148 SMs); rows sampled in the first tiles and in
+    # the tiles of the last wave
+    rows = [(0, 8), (5000, 5008), (n - 640, n - 632), (n - 8, n)]
+    err = _run(n, k, 512, rows=rows, seed=4)
+    assert err < TOL, err
