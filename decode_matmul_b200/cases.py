@@ -1,6 +1,6 @@
 """Single-kernel cases for timing and profiling (one op, seeded inputs).
 
-    python -m decode_matmul_b200.cases gemv --n 32768 --k 16384 [--reps 10]
+    python -m decode_matmul_b200.cases gemv --n 32768 --k 16384 [--reps 10] [--flush]
     python -m decode_matmul_b200.cases gemm --n 19456 --k 2560 --m 512 [--reps 10]
     python -m decode_matmul_b200.cases rht  --m 512 --k 9728 [--reps 10]
     python -m decode_matmul_b200.cases encode --n 4096 --k 14336 [--refits 0] [--reps 5]
@@ -39,6 +39,11 @@ def main(argv=None):
     ap.add_argument("--k", type=int, default=16384)
     ap.add_argument("--m", type=int, default=1)
     ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--flush", action="store_true",
+                    help="time each launch alone, after writing 256 MB (twice the L2) between launches")
+    ap.add_argument("--graph", action="store_true",
+                    help="time launches replayed from a CUDA graph (no host launch cost); with --flush, a "
+                         "graph of (256 MB write + launch) minus a graph of the writes alone")
     a = ap.parse_args(argv)
     dev = torch.device("cuda", 0)
 
@@ -93,14 +98,48 @@ def main(argv=None):
         run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.reps):
-        run()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / a.reps
+    if a.graph:
+        scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if a.flush else None
+
+        def graph_ms(with_run):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(a.reps):
+                    if scrub is not None:
+                        scrub.fill_(i & 0xFF)
+                    if with_run:
+                        run()
+            g.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / a.reps
+
+        ms = graph_ms(True) - (graph_ms(False) if a.flush else 0.0)
+    elif a.flush:
+        # each launch timed on its own (median), after the L2 has been overwritten
+        scrub = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        times = []
+        for i in range(a.reps):
+            scrub.fill_(i & 0xFF)
+            e0.record()
+            run()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+    else:
+        e0.record()
+        for _ in range(a.reps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / a.reps
     rate = work / (ms * 1e-3)
-    print(f"{a.op} n={a.n} k={a.k} m={a.m}: {ms * 1e3:.2f} us/launch, "
+    how = (" (graph" + (", L2 flushed" if a.flush else "") + ")") if a.graph else (" (L2 flushed, median)" if a.flush else "")
+    print(f"{a.op} n={a.n} k={a.k} m={a.m}{how}: {ms * 1e3:.2f} us/launch, "
           f"{rate / 1e9:.1f} G{unit}/s ({work:.4g} {unit} per launch)")
     if a.op == "ldlq":
         # the same matrix without feedback, to split the time, and the proxy loss

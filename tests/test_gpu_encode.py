@@ -169,3 +169,24 @@ def test_ldlq_full_size_sampled_rows(tq, torch_cuda):
     for r in (0, 511, 1023):
         _assert_same((codes[r:r + 1], scales[r:r + 1], err[r:r + 1]), oracle.ldlq32(w[r:r + 1], u, cb, g, 1))
 
+
+
+def test_encode_and_ldlq_without_error_output(tq, torch_cuda):
+    # err_d = NULL: the same codes and scales, nothing else written
+    import torch
+    n, k = 9, 1024
+    cb = tqsynth.codebook(20)
+    g = _gain(cb)
+    w = tqsynth.weight_rows_f32(21, n, k)
+    u = tqsynth.hessian_factor(22, k, 0.5)
+    w_d = torch.from_numpy(w).cuda()
+    u_d = torch.from_numpy(u).cuda()
+    cbd = to_dev_u16(cb.reshape(-1))
+    c1, s1, e1 = tq.tq_encode(w_d, cbd, g, 1, want_err=False)
+    c2, s2, e2 = tq.tq_ldlq_encode(w_d, u_d, cbd, g, 1, want_err=False)
+    torch.cuda.synchronize()
+    assert e1 is None and e2 is None
+    wc, ws, _ = oracle.encode32(w, cb, g, 1)
+    assert np.array_equal(c1.cpu().numpy(), wc) and np.array_equal(s1.cpu().numpy().view(np.uint16), ws)
+    lc, ls, _ = oracle.ldlq32(w, u, cb, g, 1)
+    assert np.array_equal(c2.cpu().numpy(), lc) and np.array_equal(s2.cpu().numpy().view(np.uint16), ls)
