@@ -29,7 +29,6 @@ namespace tq {
 
 constexpr int UM_BM = 128;
 constexpr int UM_BK = 64;
-constexpr int UM_STAGES = 4;
 constexpr int UM_DEC_THREADS = 256;             // 8 decoder warps: 2 threads per row
 constexpr int UM_THREADS = 128 + UM_DEC_THREADS;
 constexpr int UM_TIMEOUT_STATUS = 7;  // TQ_ERR_TIMEOUT
@@ -144,15 +143,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 template <int BN>
 struct UmmaSmem {
+  // 4 stages; the codebook as 4 views (64 KB) where that still fits (64 and
+  // 128 tokens), a single copy at 256 tokens (3 stages + 4 views measured
+  // slower there than 4 stages + one copy)
+  static constexpr int STAGES = 4;
+  static constexpr int LV = BN == 256 ? 0 : 2;
   static constexpr uint32_t A_BYTES = UM_BM * 128;     // 16 KB per stage
   static constexpr uint32_t B_BYTES = BN * 128;        // BN rows of 64 fp16
   static constexpr uint32_t C_BYTES = UM_BM * 16;      // 16 code bytes per row
   static constexpr uint32_t A_OFF = 0;
-  static constexpr uint32_t B_OFF = A_OFF + UM_STAGES * A_BYTES;
-  static constexpr uint32_t C_OFF = B_OFF + UM_STAGES * B_BYTES;
-  static constexpr uint32_t CB_OFF = C_OFF + UM_STAGES * C_BYTES;
-  static constexpr uint32_t BAR_OFF = CB_OFF + 16384;  // full[S], decoded[S], empty[S], accum
-  static constexpr uint32_t MISC_OFF = BAR_OFF + (3 * UM_STAGES + 1) * 8;
+  static constexpr uint32_t B_OFF = A_OFF + STAGES * A_BYTES;
+  static constexpr uint32_t C_OFF = B_OFF + STAGES * B_BYTES;
+  static constexpr uint32_t CB_OFF = C_OFF + STAGES * C_BYTES;
+  static constexpr uint32_t BAR_OFF = CB_OFF + (16384u << LV);  // full[S], decoded[S], empty[S], accum
+  static constexpr uint32_t MISC_OFF = BAR_OFF + (3 * STAGES + 1) * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 64;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // slack to align the base to 1024
 };
@@ -183,13 +187,14 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::MISC_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::MISC_OFF + 8);
   int* bcast = reinterpret_cast<int*>(sm + L::MISC_OFF + 16);
-  const uint32_t bar_full = base + L::BAR_OFF, bar_dec = bar_full + 8 * UM_STAGES,
-                 bar_empty = bar_dec + 8 * UM_STAGES, bar_acc = bar_empty + 8 * UM_STAGES;
+  constexpr int ST = L::STAGES;
+  const uint32_t bar_full = base + L::BAR_OFF, bar_dec = bar_full + 8 * ST, bar_empty = bar_dec + 8 * ST,
+                 bar_acc = bar_empty + 8 * ST;
 
   pdl_launch_dependents();
   if (tid == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < UM_STAGES; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_dec + 8 * s, UM_DEC_THREADS);
       mbar_init(bar_empty + 8 * s, 1);
@@ -197,9 +202,22 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     mbar_init(bar_acc, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  // codebook into shared memory (single copy: the decode is far from the limit here)
-  for (int e = tid; e < 2048; e += UM_THREADS)
-    reinterpret_cast<uint2*>(sm + L::CB_OFF)[e] = reinterpret_cast<const uint2*>(p.codebook)[e];
+  // codebook into shared memory as 2^LV interleaved views (entry e of view v
+  // at byte 8(e 2^LV + v)): decoder lane l reads view l % 2^LV, so with 4
+  // views the four lanes of a half-warp that share a view spread over four
+  // bank pairs (with one copy, 32 random 8-byte gathers cost ~7.7
+  // shared-memory wavefronts)
+  for (int e = tid; e < 2048; e += UM_THREADS) {
+    const uint2 ent = reinterpret_cast<const uint2*>(p.codebook)[e];
+    uint8_t* dst = sm + L::CB_OFF + (e << (3 + L::LV));
+    if (L::LV == 0) {
+      *reinterpret_cast<uint2*>(dst) = ent;
+    } else {
+#pragma unroll
+      for (int v = 0; v < (1 << L::LV); v += 2)
+        *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(ent.x, ent.y, ent.x, ent.y);
+    }
+  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
                  "r"(BN));
@@ -218,7 +236,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
       const uint32_t tx = L::B_BYTES + L::C_BYTES;
       int issued = 0;
       for (int i = 0; i < niters; ++i) {
-        const int s = i % UM_STAGES, r = i / UM_STAGES;
+        const int s = i % ST, r = i / ST;
         if (r > 0 && !mbar_wait(bar_empty + 8 * s, (r - 1) & 1, p.spin_limit)) {
           *abort_flag = 1;
           break;
@@ -231,10 +249,10 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
         issued = i + 1;
       }
       if (*abort_flag) {
-        // the copies still in flight belong to the last (up to) UM_STAGES
-        // issued stages: let them land before the CTA leaves
-        for (int i = issued - UM_STAGES < 0 ? 0 : issued - UM_STAGES; i < issued; ++i)
-          (void)mbar_wait(bar_full + 8 * (i % UM_STAGES), (i / UM_STAGES) & 1, p.spin_limit);
+        // the copies still in flight belong to the last (up to) ST issued
+        // stages: let them land before the CTA leaves
+        for (int i = issued - ST < 0 ? 0 : issued - ST; i < issued; ++i)
+          (void)mbar_wait(bar_full + 8 * (i % ST), (i / ST) & 1, p.spin_limit);
       }
     }
   } else if (warp == 1) {
@@ -242,7 +260,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     if (lane == 0) {
       const uint32_t idesc = umma_idesc(BN);
       for (int i = 0; i < niters; ++i) {
-        const int s = i % UM_STAGES, r = i / UM_STAGES;
+        const int s = i % ST, r = i / ST;
         if (*abort_flag || !mbar_wait(bar_dec + 8 * s, r & 1, p.spin_limit)) {
           *abort_flag = 1;
           break;
@@ -264,12 +282,12 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     const int h = dt >> 7;           // codes 8h .. 8h+7 of each 16-code chunk
     const int grow = min(row0 + r, p.n_total - 1);
     const uint16_t* srow = p.scales[seg] + (size_t)(grow - p.seg_row0[seg]) * blocks;
-    const uint8_t* cbs = sm + L::CB_OFF;
+    const uint8_t* cbs = sm + L::CB_OFF + ((lane & ((1 << L::LV) - 1)) << 3);
     uint32_t carry = 0;  // last code of this row in the previous k step
     uint32_t sc_next = __ldg(srow + b_lo);
     uint32_t sc2 = 0;
     for (int i = 0; i < niters; ++i) {
-      const int s = i % UM_STAGES, rr = i / UM_STAGES;
+      const int s = i % ST, rr = i / ST;
       if ((i & 3) == 0) {  // block start: state resets, scale of this block
         carry = 0;
         sc2 = sc_next | (sc_next << 16);
@@ -294,7 +312,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
           const int j = 2 * c + hh;
           const uint32_t code = ((j < 4 ? w0 : w1) >> (8 * (j & 3))) & 0xFFu;
           const uint32_t e = ((prev & 7u) << 8) | code;
-          const uint2 ent = *reinterpret_cast<const uint2*>(cbs + e * 8);
+          const uint2 ent = *reinterpret_cast<const uint2*>(cbs + (e << (3 + L::LV)));
           out[2 * hh] = hmul2_u32(ent.x, sc2);
           out[2 * hh + 1] = hmul2_u32(ent.y, sc2);
           prev = code;
