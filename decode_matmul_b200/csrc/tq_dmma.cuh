@@ -419,8 +419,11 @@ __device__ __forceinline__ void wait_xflag(const volatile int* xflag, int blk, i
 }
 
 // XCG: the small-batch activations were written earlier in the same launch
-// (persistent stack), so they are read through L2 (ld.global.cg) instead of
-// the read-only path.
+// (persistent stack), so they are read with coherent loads (ld.global.ca)
+// instead of the read-only path: the writes are released before the grid
+// barrier and acquired by the barrier's waiting thread, whose CTA barrier
+// then orders every thread's later loads after that acquire, so L1 holds no
+// stale line of them; a CTA's units reuse each block of x' across tiles.
 // A warp's partial of one tile into its shared-memory slot (16 rows x MC
 // tokens, the layout of the global partials).
 template <int NT, bool HILO>
@@ -533,7 +536,7 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
           if ((j & 1) == 0) {
 #pragma unroll
             for (int jt = 0; jt < NT; ++jt)
-              bpair[jt] = XCG ? __ldcg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j))
+              bpair[jt] = XCG ? __ldca(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j))
                               : __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j));
           }
 #pragma unroll
