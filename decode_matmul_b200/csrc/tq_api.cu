@@ -996,8 +996,14 @@ int tq_ldlq_encode(const float* w_rot_d, int32_t n, int32_t k, const float* u_d,
   cudaStream_t s = (cudaStream_t)stream;
   for (int b = 0; b < kb; ++b) {
     if (b > 0) {
-      st = launch(tq::ldlq_feedback_kernel, dim3((unsigned)((n + tq::kFbTile - 1) / tq::kFbTile), 256 / tq::kFbTile),
-                  dim3(256), 0, s, w_rot_d, (const float*)delta, u_d, (int)n, (int)k, b, wt);
+      // 64-row tiles when they give at least one per SM, else 32-row tiles
+      const bool wide = (int64_t)((n + 63) / 64) * (256 / tq::kFbCols) >= sms;
+      if (wide)
+        st = launch(tq::ldlq_feedback_kernel<4>, dim3((unsigned)((n + 63) / 64), 256 / tq::kFbCols), dim3(256), 0, s,
+                    w_rot_d, (const float*)delta, u_d, (int)n, (int)k, b, wt);
+      else
+        st = launch(tq::ldlq_feedback_kernel<2>, dim3((unsigned)((n + 31) / 32), 256 / tq::kFbCols), dim3(256), 0, s,
+                    w_rot_d, (const float*)delta, u_d, (int)n, (int)k, b, wt);
       if (st != TQ_OK) return st;
     }
     tq::EncArgs a = {};

@@ -290,23 +290,28 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(EncArgs a) {
 // each row is encoded from
 //   wt[r][j] = w[r][256b + j] + sum_{i < 256b} delta[r][i] * U[i][256b + j],
 // each element summed by fma in ascending i (binary32), delta = w - w_hat of the
-// blocks already coded.  A plain tiled SIMT GEMM: 64 x 64 outputs per CTA,
-// a 4 x 4 register tile per thread, 32-deep k tiles in shared memory; every
-// output keeps its own accumulator, so the order per output is ascending i.
-constexpr int kFbTile = 64, kFbDepth = 32;
+// blocks already coded.  A plain tiled SIMT GEMM: 16 TM x 64 outputs per CTA
+// (TM = 4, or 2 when there are too few rows to fill the GPU with 64-row
+// tiles), a TM x 4 register tile per thread, 32-deep k tiles in shared
+// memory; every output keeps its own accumulator, so the order per output is
+// ascending i.
+constexpr int kFbCols = 64, kFbDepth = 32;
 
+template <int TM>
 __global__ void __launch_bounds__(256) ldlq_feedback_kernel(const float* __restrict__ w, const float* __restrict__ delta,
                                                             const float* __restrict__ u, int n, int k, int b,
                                                             float* __restrict__ wt) {
-  __shared__ __align__(16) float As[kFbDepth][kFbTile + 4];  // delta tile, [i][row]
-  __shared__ __align__(16) float Bs[kFbDepth][kFbTile];      // U tile, [i][col]
+  constexpr int ROWS = 16 * TM;                              // rows of the CTA tile
+  constexpr int PER = ROWS * kFbDepth / 256;                 // delta values each thread stages (8 or 4)
+  __shared__ __align__(16) float As[kFbDepth][ROWS + 4];     // delta tile, [i][row]
+  __shared__ __align__(16) float Bs[kFbDepth][kFbCols];      // U tile, [i][col]
   const int tid = threadIdx.x, tr = tid >> 4, tc = tid & 15;
-  const int row0 = blockIdx.x * kFbTile, col0 = blockIdx.y * kFbTile;
+  const int row0 = blockIdx.x * ROWS, col0 = blockIdx.y * kFbCols;
   const long long cw = 256LL * b + col0 + tc * 4;  // this thread's first column in w / U
-  float acc[4][4];
+  float acc[TM][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = row0 + tr * 4 + i;
+  for (int i = 0; i < TM; ++i) {
+    const int r = row0 + tr * TM + i;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < n) v = __ldg(reinterpret_cast<const float4*>(w + (long long)r * k + cw));
     acc[i][0] = v.x;
@@ -314,44 +319,57 @@ __global__ void __launch_bounds__(256) ldlq_feedback_kernel(const float* __restr
     acc[i][2] = v.z;
     acc[i][3] = v.w;
   }
-  const int lr = tid >> 2, lk = (tid & 3) * 8;  // delta tile loads: row lr, 8 values from lk
-  const int ui = tid >> 3, uc = (tid & 7) * 8;  // U tile loads: row ui, 8 values from uc
+  const int lr = tid / (kFbDepth / PER), lk = (tid % (kFbDepth / PER)) * PER;  // delta loads: row lr, PER values
+  const int ui = tid >> 3, uc = (tid & 7) * 8;                                 // U tile loads: row ui, 8 values
   const int kend = 256 * b;
   for (int k0 = 0; k0 < kend; k0 += kFbDepth) {
-    float4 d0 = make_float4(0.f, 0.f, 0.f, 0.f), d1 = d0;
+    float dv[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) dv[e] = 0.f;
     if (row0 + lr < n) {
       const float* dp = delta + (long long)(row0 + lr) * k + k0 + lk;
-      d0 = __ldg(reinterpret_cast<const float4*>(dp));
-      d1 = __ldg(reinterpret_cast<const float4*>(dp + 4));
+#pragma unroll
+      for (int e = 0; e < PER; e += 4) {
+        const float4 d4 = __ldg(reinterpret_cast<const float4*>(dp + e));
+        dv[e] = d4.x;
+        dv[e + 1] = d4.y;
+        dv[e + 2] = d4.z;
+        dv[e + 3] = d4.w;
+      }
     }
     const float* up = u + (long long)(k0 + ui) * k + 256LL * b + col0 + uc;
     const float4 u0 = __ldg(reinterpret_cast<const float4*>(up)), u1 = __ldg(reinterpret_cast<const float4*>(up + 4));
-    As[lk + 0][lr] = d0.x;
-    As[lk + 1][lr] = d0.y;
-    As[lk + 2][lr] = d0.z;
-    As[lk + 3][lr] = d0.w;
-    As[lk + 4][lr] = d1.x;
-    As[lk + 5][lr] = d1.y;
-    As[lk + 6][lr] = d1.z;
-    As[lk + 7][lr] = d1.w;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) As[lk + e][lr] = dv[e];
     *reinterpret_cast<float4*>(&Bs[ui][uc]) = u0;
     *reinterpret_cast<float4*>(&Bs[ui][uc + 4]) = u1;
     __syncthreads();
 #pragma unroll 8
     for (int kk = 0; kk < kFbDepth; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[kk][tr * 4]);
+      float a4[TM];
+      if (TM == 4) {
+        const float4 av = *reinterpret_cast<const float4*>(&As[kk][tr * 4]);
+        a4[0] = av.x;
+        a4[1] = av.y;
+        a4[2 % TM] = av.z;
+        a4[3 % TM] = av.w;
+      } else {
+        const float2 av = *reinterpret_cast<const float2*>(&As[kk][tr * 2]);
+        a4[0] = av.x;
+        a4[1] = av.y;
+      }
       const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tc * 4]);
-      const float a4[4] = {av.x, av.y, av.z, av.w}, b4[4] = {bv.x, bv.y, bv.z, bv.w};
+      const float b4[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < TM; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = row0 + tr * 4 + i;
+  for (int i = 0; i < TM; ++i) {
+    const int r = row0 + tr * TM + i;
     if (r < n)
       *reinterpret_cast<float4*>(wt + (long long)r * 256 + col0 + tc * 4) =
           make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);

@@ -190,3 +190,15 @@ def test_encode_and_ldlq_without_error_output(tq, torch_cuda):
     assert np.array_equal(c1.cpu().numpy(), wc) and np.array_equal(s1.cpu().numpy().view(np.uint16), ws)
     lc, ls, _ = oracle.ldlq32(w, u, cb, g, 1)
     assert np.array_equal(c2.cpu().numpy(), lc) and np.array_equal(s2.cpu().numpy().view(np.uint16), ls)
+
+
+def test_ldlq_wide_feedback_tiles(tq, torch_cuda):
+    # enough rows for the 64-row feedback tiles (n >= 4736 on 148 SMs); sampled rows bit-exact
+    n, k = 4800, 1024
+    cb = tqsynth.codebook(23)
+    g = _gain(cb)
+    w = tqsynth.weight_rows_f32(24, n, k)
+    u = tqsynth.hessian_factor(25, k, 0.5)
+    codes, scales, err = _gpu_ldlq(tq, torch_cuda, w, u, cb, g, 0)
+    for r in (0, 63, 64, 2399, 4799):
+        _assert_same((codes[r:r + 1], scales[r:r + 1], err[r:r + 1]), oracle.ldlq32(w[r:r + 1], u, cb, g, 0))
