@@ -478,6 +478,40 @@ def test_hessian_factor_is_block_strictly_upper():
 
 # ---- stack -------------------------------------------------------------------------------
 
+@pytest.mark.parametrize("p", [0, 2])
+def test_stack_phase_constant_codebook_closed_form(p):
+    # Every codebook entry 1 and one scale per row: W[n][k] = s_n, and the
+    # Sylvester Hadamard's columns sum to 0 except the first, so each 512-block
+    # of x' sums to sqrt(512) d_0 x_0 and y_n = s_n sqrt(512) sum_B d_512B x_512B.
+    # Pins the phase composition: the RHT seed, every op of the phase, and
+    # which op feeds the bf16 handoff with which alpha.
+    m, k = 2, 1024
+    seed = 4242
+    cb = np.full(8 * 256 * 4, np.float16(1.0).view(np.uint16), dtype=np.uint16)
+    rng = np.random.default_rng(p)
+    ops = oracle.PHASES[p]
+    weights = {}
+    for i, op in enumerate(ops):
+        n = 48 + 16 * i
+        s_row = (0.005 + 0.025 * rng.random(n)).astype(np.float16)
+        scales = np.repeat(s_row.view(np.uint16)[:, None], k // 256, axis=1)
+        codes = rng.integers(0, 256, size=(n, k // 4), dtype=np.uint8)
+        weights[op] = (codes, scales, cb, n, k)
+    x = tqsynth.activations(p + 7, m, k)
+    ys, hand = oracle.stack_phase(p, x, m, weights, seed)
+    d = oracle.rht_signs(seed, k).astype(np.float64)
+    xv = tqsynth.bf16_to_f64(x)
+    col = (xv[:, ::512] * d[::512]).sum(axis=1) * math.sqrt(512.0)  # [m]
+    for op in ops:
+        s_row = tqsynth.f16_to_f64(weights[op][1][:, 0])
+        want = col[:, None] * s_row[None, :]
+        assert np.allclose(ys[op], want, rtol=1e-12, atol=1e-15)
+    hop = oracle.HANDOFF_OP[p]
+    assert hop == ops[0]
+    want_h = tqsynth.bf16_bits(oracle.alpha(k) * ys[hop])
+    assert np.array_equal(hand, want_h)
+
+
 def test_alpha_second_moment_closed_form():
     a, b = oracle.SCALE_LO, oracle.SCALE_HI
     assert abs(oracle.E_S2 - (a * a + a * b + b * b) / 3) < 1e-18
