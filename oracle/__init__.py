@@ -17,7 +17,7 @@ Pages (cited by title and section):
   * "8 open models ... what 2-bit quantization costs", "Size": per-block
     scales add bits on top of the 2-bit codes.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * layout: codes uint8 [n][k/4]; state = previous code & 7, reset every
     256 weights; fp16 scale per (row, 256-block); codebook fp16 [8][256][4];
     component j of an entry is weight 4g+j.
