@@ -81,8 +81,39 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.nvml = []           # (time, SM MHz, max SM MHz, reason bits) from the polling thread
+        self.window = None       # (t0, t1) of the timed region, time.perf_counter()
+        self._stop = None
+        self._thread = None
+
+    def _poll_nvml(self):
+        # NVML reads only (no setting is changed); ~1 ms between samples so that
+        # a timed region of a few tens of ms still gets many
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self._stop.is_set():
+                self.nvml.append((time.perf_counter(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx,
+                                  reasons(h)))
+                time.sleep(0.001)
+            pynvml.nvmlShutdown()
+        except Exception:  # no NVML: the nvidia-smi samples stand
+            pass
+
+    def mark(self, t0: float, t1: float):
+        """The timed region (time.perf_counter() before its first launch and
+        after its synchronize)."""
+        self.window = (t0, t1)
 
     def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        self._thread.start()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -92,6 +123,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *a):
+        if self._stop is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
         self.lines = []
         if self.proc is not None:
             self.proc.terminate()
@@ -102,7 +136,17 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
+    # NVML clock-event reason bits
+    NVML_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
+
     def summary(self):
+        if self.window is not None:
+            t0, t1 = self.window
+            inside = [x for x in self.nvml if t0 <= x[0] <= t1]
+            if inside:
+                reasons = sorted(n for n, bit in self.NVML_BITS.items() if any(x[3] & bit for x in inside))
+                return {"sm_mhz": float(np.median([x[1] for x in inside])), "sm_max_mhz": float(inside[0][2]),
+                        "reasons": reasons, "samples": len(inside), "source": "nvml, timed region"}
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in getattr(self, "lines", []):
@@ -119,7 +163,8 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvidia-smi"}
 
 
 # ---- stack construction ----------------------------------------------------------
@@ -344,12 +389,14 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         time.sleep(0.3)  # sampler start-up
+        t_start = time.perf_counter()
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(args.steps):
                 graph.replay()
             e1.record(stream)
         stream.synchronize()
+        clk.mark(t_start, time.perf_counter())
     torch.cuda.synchronize()
     barrier()
     ms = e0.elapsed_time(e1) / args.steps
