@@ -27,3 +27,22 @@ def test_reference_arm_prints_one_contract_line():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_clock_summary_keeps_the_timed_region_only():
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.ClockSampler(0)
+    # (time, SM MHz, max MHz, reason bits): idle samples outside the window
+    c.nvml = [(0.0, 345, 1965, 0), (1.0, 1965, 1965, 0), (1.1, 1965, 1965, 0x4), (1.2, 1950, 1965, 0),
+              (5.0, 300, 1965, 0x8)]
+    c.mark(0.9, 1.3)
+    s = c.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["source"].startswith("nvml")
+    # without NVML samples in the window: the nvidia-smi lines
+    c2 = bench.ClockSampler(0)
+    c2.lines = ["0, 1965, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Active",
+                "0, 1900, 1965, 710.0, 0x4, Not Active, Not Active, Not Active, Active"]
+    s2 = c2.summary()
+    assert s2["samples"] == 2 and s2["reasons"] == ["sw_power_cap"] and s2["source"] == "nvidia-smi"
