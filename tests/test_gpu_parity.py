@@ -108,7 +108,7 @@ def test_gemv_deterministic_and_counters_reset(tq, torch_cuda):
 
 # ---- small-batch GEMM -------------------------------------------------------------
 
-@pytest.mark.parametrize("m", [2, 7, 8, 16, 33, 64, 100])
+@pytest.mark.parametrize("m", [2, 7, 8, 16, 17, 24, 31, 33, 64, 100])
 def test_gemm_small_batch(tq, torch_cuda, m):
     import torch
     n, k = 1040, 1536
@@ -163,7 +163,7 @@ def _check_handoff(h_bits, y_gpu, hand_oracle, k):
     assert np.all(np.abs(got - want) <= step + TOL * np.maximum(np.abs(want), rms))
 
 
-@pytest.mark.parametrize("m", [1, 3])
+@pytest.mark.parametrize("m", [1, 3, 20])
 def test_layer_phases_teacher_forced(tq, torch_cuda, m):
     import torch
     hl = _host_layers(SMALL)
