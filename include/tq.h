@@ -290,8 +290,10 @@ TQ_API int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t*
  *           strictly upper part is read).
  * err_d:    device fp32 [n][k/256] or NULL: per block, the fold-order sum of
  *           (w~ - w_hat)^2.
- * workspace_d: device, >= tq_ldlq_workspace bytes, 16-byte aligned (E and
- *           the adjusted block; no initial contents needed).
+ * workspace_d: device, >= tq_ldlq_workspace bytes = 4 n (k + 256), 16-byte
+ *           aligned (E and the adjusted block; no initial contents needed).
+ * Errors: those of tq_encode; TQ_ERR_NULL for a NULL u_d; TQ_ERR_ALIGN for
+ * u_d or workspace_d; TQ_ERR_WORKSPACE for a missing or short workspace.
  * Enqueues 2*(k/256) - 1 launches on `stream`. */
 TQ_API int tq_ldlq_workspace(int32_t n, int32_t k, size_t* bytes);
 TQ_API int tq_ldlq_encode(const float* w_rot_d, int32_t n, int32_t k, const float* u_d, const uint16_t* codebook_d,
