@@ -478,7 +478,7 @@ def test_hessian_factor_is_block_strictly_upper():
 
 # ---- stack -------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("p", [0, 2])
+@pytest.mark.parametrize("p", [0, 1, 2, 3])
 def test_stack_phase_constant_codebook_closed_form(p):
     # Every codebook entry 1 and one scale per row: W[n][k] = s_n, and the
     # Sylvester Hadamard's columns sum to 0 except the first, so each 512-block
@@ -510,6 +510,67 @@ def test_stack_phase_constant_codebook_closed_form(p):
     assert hop == ops[0]
     want_h = tqsynth.bf16_bits(oracle.alpha(k) * ys[hop])
     assert np.array_equal(hand, want_h)
+
+
+def _signs_from_definition(seed_lp: int, k: int) -> np.ndarray:
+    """d[j] = -1 when the top bit of the j-th SplitMix64 output (state seed_lp)
+    is set, from the input generator's SplitMix64 (not the oracle's)."""
+    return np.where(tqsynth.draws(seed_lp, 0, k) >> np.uint64(63), -1.0, 1.0)
+
+
+def _phase_seed_from_definition(seed: int, l: int, p: int) -> int:
+    return tqsynth.mix64_int(seed ^ tqsynth.mix64_int(0x516E0000 | (l << 2) | p))
+
+
+def test_layer_stack_constant_codebook_closed_form_chain():
+    # Three layers with every codebook entry 1 and one fp16 scale per row.
+    # Then W = s_n, each phase's outputs are y_n = s_n * c with
+    # c = sqrt(512) * sum_B d[512B] x[512B] (x = the phase input, d = that
+    # phase's signs), and the whole stack collapses to a scalar recurrence on
+    # the handoff op's row scales.  A wrong per-(layer, phase) seed, a phase
+    # reading the wrong input, the wrong op handed on, or alpha of the wrong
+    # width changes the chain.
+    m, seed = 2, 987654321
+    hidden, q, kv, inter = 1024, 512, 512, 1536
+    shape = tqsynth.StackShape("chain", 3, hidden, q, kv, inter)
+    cb = np.full((8, 256, 4), np.float16(1.0).view(np.uint16), dtype=np.uint16)
+    rng = np.random.default_rng(77)
+    layers = []
+    for _ in range(shape.layers):
+        w = {}
+        for op, n, k in shape.ops():
+            s_row = (0.005 + 0.025 * rng.random(n)).astype(np.float16).view(np.uint16)
+            scales = np.repeat(s_row[:, None], k // 256, axis=1)
+            codes = rng.integers(0, 256, size=(n, k // 4), dtype=np.uint8)
+            w[op] = (codes, scales, cb, n, k)
+        layers.append(w)
+    x = tqsynth.activations(55, m, hidden)
+    h_out, trace = oracle.layer_stack(layers, x, m, seed)
+    assert len(trace) == 4 * shape.layers
+
+    handoff_op = {0: "q", 1: "o", 2: "gate", 3: "down"}
+    h = tqsynth.bf16_to_f64(x)  # [m][k] values of the current phase input
+    f = 0
+    for l, w in enumerate(layers):
+        for p in range(4):
+            op = handoff_op[p]
+            n, k = w[op][3], w[op][4]
+            assert k == h.shape[1]
+            d = _signs_from_definition(_phase_seed_from_definition(seed, l, p), k)
+            c = math.sqrt(512.0) * (h[:, ::512] * d[::512]).sum(axis=1)  # [m]
+            s_row = tqsynth.f16_to_f64(w[op][1][:, 0])
+            a = 1.0 / math.sqrt(k * (0.03 ** 3 - 0.005 ** 3) / (3 * 0.025))
+            want = tqsynth.bf16_bits(a * (c[:, None] * s_row[None, :]))
+            assert np.array_equal(trace[f], want), (l, p)
+            h = tqsynth.bf16_to_f64(want)
+            f += 1
+    assert np.array_equal(h_out, trace[-1])
+
+
+def test_stack_phase_seeds_differ_per_layer_and_phase():
+    seeds = {oracle.stack_phase_seed(3, l, p) for l in range(8) for p in range(4)}
+    assert len(seeds) == 32
+    assert oracle.stack_phase_seed(3, 2, 1) == _phase_seed_from_definition(3, 2, 1)
 
 
 def test_alpha_second_moment_closed_form():
