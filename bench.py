@@ -12,8 +12,12 @@ no L2 flush is needed between steps.
 
 Prints ONE JSON line on rank 0.  N > 1 (torchrun) runs N independent replicas
 (the path has no exchange step): value = all ranks' tokens / max-over-ranks time.
-`--impl reference` times the CPU oracle (fp64 C, one host core) on a bounded
-sample of the same workload.
+The line also carries `gemv`: the batch-1 decode-GEMV alone (tq_gemv on a
+32768 x 16384 weight, two copies read in turn so no launch finds its weight in
+L2), the first half of the metric, with its own roofline and clocks.
+`--impl reference` times the CPU oracle (fp64 C, on all host cores) on a
+bounded sample of the same workload; our arm's `cpu_baseline` is the same
+recipe, on all cores and on one.
 """
 from __future__ import annotations
 
@@ -199,72 +203,132 @@ def phase_bytes(shape, m):
     return out
 
 
+STACK_SOURCES = ("tq_common.cuh", "tq_rht.cuh", "tq_dmma.cuh", "tq_stack1.cuh")
+
+
+def kernel_source_hash(names=STACK_SOURCES) -> str:
+    """sha256 over the CUDA sources of a kernel (to tell whether an ncu figure
+    was taken on the kernel that runs now)."""
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "decode_matmul_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def ncu_traffic(shape_name, layers, m):
-    """DRAM bytes (read + write) per launch of the batch-1 stack kernel, from the
-    committed ncu summary of the Qwen3-4B-shaped stack (measured on 6 layers,
-    scaled per layer); None for any other shape or batch (not captured)."""
-    p = os.path.join(ROOT, "profiles", "stack1_kernel_qwen3-4b-shaped_m1.md")
-    if m != 1 or shape_name != "qwen3-4b-shaped" or not os.path.exists(p):
+    """DRAM bytes (read + write) per launch of the batch-1 stack kernel from
+    the ncu figure stored in profiles/ (measured on a few layers, scaled by
+    layers: every layer has the same shapes), or None when there is no figure
+    for this shape and batch or the kernel's sources changed since it was
+    taken."""
+    p = os.path.join(ROOT, "profiles", "stack1_kernel_traffic.json")
+    if m != 1 or not os.path.exists(p):
         return None
     with open(p) as f:
-        for ln in f:
-            if ln.startswith("dram_bytes_per_layer:"):
-                return float(ln.split(":")[1]) * layers
-    return None
+        d = json.load(f)
+    if d.get("workload") != shape_name or d.get("source_sha256") != kernel_source_hash():
+        return None
+    return float(d["dram_bytes_per_layer"]) * layers
 
 
-# ---- reference arm (CPU oracle) ---------------------------------------------------
+# ---- the CPU oracle on a bounded sample (reference arm and cpu_baseline) ---------------
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_layer_sample(shape, m, frac, threads, layer=0, seed=0):
+    """One layer of the stack on the oracle, sampled: per phase one RHT of a
+    seeded bf16 input of the phase's width with that layer's phase seed, then
+    the first round(frac * n) rows of every op of the phase (decode + fp64
+    matmul), split over `threads` host threads (the C oracle releases the GIL).
+    Returns (seconds spent, the same scaled to every row of the layer, rows
+    done)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    cb = tqsynth.codebook(seed)
+    ops = shape.ops()
+    opi = {op: i for i, (op, _, _) in enumerate(ops)}
+    dims = {op: (n, k) for op, n, k in ops}
+    t_all = t_full = 0.0
+    done = 0
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for p, group in enumerate(oracle.PHASES):
+            k = dims[group[0]][1]
+            x = tqsynth.activations(seed, m, k, stream=p + 1)
+            data = []
+            for op in group:
+                n = dims[op][0]
+                r = max(1, min(n, int(round(frac * n))))
+                data.append((op, n, r, tqsynth.codes_rows(seed, layer, opi[op], k, 0, r),
+                             tqsynth.scales(seed, layer, opi[op], r, k)))
+            ts = time.perf_counter()
+            xr = oracle.rht(x, m, k, oracle.stack_phase_seed(seed, layer, p))
+            t_rht = time.perf_counter() - ts
+            t_phase_full = t_rht
+            for op, n, r, c, sc in data:
+                ts = time.perf_counter()
+                chunks = [(i * r // threads, (i + 1) * r // threads) for i in range(threads)]
+                list(ex.map(lambda ab: oracle.linear_rows(c, sc, cb, k, xr, m, ab[0], ab[1]) if ab[1] > ab[0]
+                            else None, chunks))
+                t = time.perf_counter() - ts
+                t_phase_full += t * n / r
+                t_all += t
+                done += r
+            t_all += t_rht
+            t_full += t_phase_full
+    return t_all, t_full, done
+
+
+def oracle_sample_frac(shape, m, budget_s, threads):
+    """Fraction of each op's rows whose oracle run takes about budget_s on
+    `threads` threads (from a 2-row probe of every op, single-threaded)."""
+    import oracle
+    oracle.build()
+    _, t_layer_1, _ = oracle_layer_sample(shape, m, 0.0, 1)  # 1 row of each op -> full-layer estimate
+    t_layer_par = t_layer_1 / max(1, threads)
+    return min(1.0, budget_s / max(t_layer_par, 1e-9))
+
+
+def oracle_baseline(shape, m, budget_s=8.0):
+    """The oracle timed on the host's cores: the same sample run on all host
+    cores and on one; tokens/s of the whole stack extrapolated from it."""
+    cores = host_cores()
+    frac = oracle_sample_frac(shape, m, budget_s, cores)
+    t_par, full_par, rows = oracle_layer_sample(shape, m, frac, cores)
+    t_one, full_one, _ = oracle_layer_sample(shape, m, frac, 1)
+    full_rows = sum(n for _, n, _ in shape.ops())
+    sample = (f"{rows} of the {full_rows} weight rows of layer 0 (the same fraction of each of its 7 ops, "
+              f"with the 4 RHTs of that layer's phase seeds), m={m}; each op's time scaled by its row count, then "
+              f"to {shape.layers} layers; {t_par:.1f} s on {cores} threads, {t_one:.1f} s on 1")
+    return {"value": m / (full_par * shape.layers), "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": sample, "single_thread_value": m / (full_one * shape.layers), "host_cores": cores}
+
 
 def run_reference(args, shape, m):
     import oracle
     oracle.build()
-    seed = 0
     steps, warm = args.steps, args.warmup
+    cores = host_cores()
     # per-step CPU budget so that warmup + steps end in about two minutes
     budget = max(2.0, 120.0 / max(1, steps + warm))
-    ops = shape.ops()
-    x = tqsynth.activations(seed, m, shape.hidden)
-    cb = tqsynth.codebook(seed)
-    # rows of each op in the sample: the same fraction f of every op of layer 0
-    t0 = time.perf_counter()
-    probe_rows = 4
-    for i, (op, n, k) in enumerate(ops):
-        c = tqsynth.codes_rows(seed, 0, i, k, 0, probe_rows)
-        s = tqsynth.scales(seed, 0, i, probe_rows, k)
-        xr = np.zeros((m, k))
-        oracle.linear_rows(c, s, cb, k, xr, m, 0, probe_rows)
-    per_row_layer = (time.perf_counter() - t0) / probe_rows  # one row of every op
-    rows = max(1, min(min(n for _, n, _ in ops), int(budget / max(per_row_layer, 1e-9))))
-    frac = {op: rows / n for op, n, _ in ops}
-
-    def one_step():
-        h = x
-        ts = time.perf_counter()
-        for p, group in enumerate(oracle.PHASES):
-            k = dict((o, kk) for o, _, kk in ops)[group[0]]
-            xr = oracle.rht(h if h.shape[1] == k else tqsynth.activations(seed + 1 + p, m, k), m, k,
-                            oracle.stack_phase_seed(seed, 0, p))
-            for op in group:
-                i = [o for o, _, _ in ops].index(op)
-                n = [nn for o, nn, _ in ops if o == op][0]
-                r = max(1, int(round(frac[op] * n)))
-                c = tqsynth.codes_rows(seed, 0, i, k, 0, r)
-                s = tqsynth.scales(seed, 0, i, r, k)
-                oracle.linear_rows(c, s, cb, k, xr, m, 0, r)
-        return time.perf_counter() - ts
-
+    frac = oracle_sample_frac(shape, m, budget, cores)
     for _ in range(warm):
-        one_step()
-    times = [one_step() for _ in range(steps)]
-    t_step = float(np.mean(times))
-    # the sample is `rows` rows of every op of one layer: scale to the whole stack
-    full_rows = sum(n for _, n, _ in ops)
-    sample_rows = sum(max(1, int(round(frac[op] * n))) for op, n, _ in ops)
-    t_token = t_step * (full_rows / sample_rows) * shape.layers / m
+        oracle_layer_sample(shape, m, frac, cores)
+    runs = [oracle_layer_sample(shape, m, frac, cores) for _ in range(steps)]
+    t_step = float(np.mean([r[0] for r in runs]))
+    t_token = float(np.mean([r[1] for r in runs])) * shape.layers / m
     value = 1.0 / t_token
-    sample = (f"{sample_rows} of {full_rows} weight rows of layer 0 (all 7 ops, all 4 RHTs) at m={m}, "
-              f"scaled by rows and by {shape.layers} layers")
-    cpu = {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle", "sample": sample}
+    full_rows = sum(n for _, n, _ in shape.ops())
+    sample = (f"{runs[0][2]} of the {full_rows} weight rows of layer 0 (the same fraction of each of its 7 ops, "
+              f"with the 4 RHTs of that layer's phase seeds) at m={m} per step on {cores} threads, scaled by rows "
+              f"and by {shape.layers} layers")
+    cpu = {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
             "steps": steps, "warmup": warm, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -275,51 +339,64 @@ def run_reference(args, shape, m):
     print(json.dumps(line), flush=True)
 
 
-# ---- our arm ------------------------------------------------------------------------
+# ---- the batch-1 decode-GEMV on its own (first half of the metric) --------------------
 
-def cpu_baseline_quick(shape, m):
-    """The oracle on ~10-20 s of host work: the same fraction of the rows of
-    each op of layer 0 (with its RHT), each op's time scaled by its row count,
-    summed, and scaled to the whole stack."""
-    import oracle
-    oracle.build()
-    seed = 0
-    cb = tqsynth.codebook(seed)
-    ops = shape.ops()
-    t_target = 12.0
-    cost = []  # seconds per row of each op (2-row probe)
-    for i, (op, n, k) in enumerate(ops):
-        c = tqsynth.codes_rows(seed, 0, i, k, 0, 2)
-        s = tqsynth.scales(seed, 0, i, 2, k)
+GEMV_SHAPE = (32768, 16384)  # 138 MB packed: larger than the 126 MB L2 on its own
+GEMV_COPIES = 2              # distinct weights read in turn: 277 MB per round
+
+
+def bench_gemv(tq, dev, stream, steps, warmup, hbm):
+    """tq_gemv on GEMV_COPIES distinct n x k weights in turn, launches replayed
+    from a CUDA graph; each launch reads a weight the previous launch did not
+    touch, and the copies together are twice the L2, so no launch starts with
+    its weight in L2.  Returns the JSON object (GB/s over algorithmic bytes)."""
+    import torch
+    n, k = GEMV_SHAPE
+    ws = []
+    for c in range(GEMV_COPIES):
+        ws.append(tq.DeviceWeight.from_host(tqsynth.codes(0, 100 + c, 0, n, k), tqsynth.scales(0, 100 + c, 0, n, k),
+                                            tqsynth.codebook(0), n, k, device=dev))
+    x = torch.from_numpy(tqsynth.bf16_to_f64(tqsynth.activations(0, 1, k))[0].astype(np.float32)).to(dev)
+    y = torch.empty(n, dtype=torch.float32, device=dev)
+    wsp = tq.workspace(tq.tq_gemv_workspace(n, k), dev)
+    per_graph = 2 * GEMV_COPIES
+    with torch.cuda.stream(stream):
+        for i in range(per_graph):
+            tq.tq_gemv(ws[i % GEMV_COPIES], x, y, wsp, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(per_graph):
+            tq.tq_gemv(ws[i % GEMV_COPIES], x, y, wsp, stream=stream)
+    reps = max(3, steps)
+    for _ in range(max(3, warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        time.sleep(0.3)
         t0 = time.perf_counter()
-        oracle.linear_rows(c, s, cb, k, np.zeros((m, k)), m, 0, 2)
-        cost.append((time.perf_counter() - t0) / 2)
-    t_est = sum(n * c for (_, n, _), c in zip(ops, cost))  # one whole layer
-    frac = min(1.0, t_target / max(t_est, 1e-9))
-    n_layers = max(1, min(shape.layers, int(round(t_target / max(t_est, 1e-9))))) if frac >= 1.0 else 1
-    x = tqsynth.activations(seed, m, shape.hidden)
-    t_layers, t_all, done = 0.0, 0.0, 0
-    for l in range(n_layers):
-        for i, (op, n, k) in enumerate(ops):
-            rows = max(1, min(n, int(round(frac * n))))
-            xin = x if k == shape.hidden else tqsynth.activations(seed + 1 + i, m, k)
-            c = tqsynth.codes_rows(seed, l, i, k, 0, rows)
-            s = tqsynth.scales(seed, l, i, rows, k)
-            ts = time.perf_counter()
-            xr = oracle.rht(xin, m, k, oracle.stack_phase_seed(seed, l, 0))
-            oracle.linear_rows(c, s, cb, k, xr, m, 0, rows)
-            t = time.perf_counter() - ts
-            t_all += t
-            t_layers += t * n / rows
-            done += rows
-    full_rows = sum(n for _, n, _ in ops)
-    t_token = t_layers / n_layers * shape.layers / m
-    what = (f"all {full_rows} rows of layers 0-{n_layers - 1}" if frac >= 1.0 else
-            f"{done} of the {full_rows} rows of layer 0 (the same fraction of each of its 7 ops)")
-    return {"value": 1.0 / t_token, "unit": "tok/s", "cores": 1, "kind": "oracle",
-            "sample": f"{what} with their RHTs, m={m}, {t_all:.1f} s single-threaded, each op scaled by its "
-                      f"row count, then to {shape.layers} layers"}
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        clk.mark(t0, time.perf_counter())
+    us = e0.elapsed_time(e1) * 1e3 / (reps * per_graph)
+    packed = tqsynth.pack_bytes(n, k)
+    alg = packed + 16384 + 4 * k + 4 * n  # codes + scales, codebook, x' fp32, y fp32
+    gbs = alg / (us * 1e-6) / 1e9
+    return {"workload": f"one {n} x {k} trellis-coded weight ({packed / 1e6:.1f} MB packed), batch 1, "
+                        f"{GEMV_COPIES} distinct copies read in turn ({GEMV_COPIES * packed / 1e6:.0f} MB > 126 MB L2)",
+            "kernel": "dmma_kernel<LV=3, hilo> (tq_gemv: register decode + mma.sync)",
+            "us_per_launch": us, "launches": reps * per_graph, "compressed_weight_gbs": packed / (us * 1e-6) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "bytes_per_launch": alg},
+            "clocks": clk.summary()}
 
+
+# ---- our arm ------------------------------------------------------------------------
 
 def main():
     ap = argparse.ArgumentParser()
@@ -331,6 +408,7 @@ def main():
     ap.add_argument("--m", type=int, default=None)
     ap.add_argument("--layers", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gemv", action="store_true", help="skip the stand-alone decode-GEMV measurement")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -461,9 +539,12 @@ def main():
     e2e_ms = ee0.elapsed_time(ee1) / args.steps
     e2e_val = replica_throughput(m, world, 1, max_over_ranks(e2e_ms, dist, dev))
 
+    # the decode-GEMV on its own (every rank runs it on its own GPU; rank 0 reports)
+    gemv = None if args.no_gemv else bench_gemv(tq, dev, stream, args.steps, args.warmup, measured_peaks()[0])
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_quick(shape, m)
+        cpu = oracle_baseline(shape, m)
 
     if dist is not None:
         del graph
@@ -506,6 +587,7 @@ def main():
         "e2e": {"value": e2e_val, "unit": "tok/s", "h2d_bytes_per_step": int(h_host.numel() * 2),
                 "d2h_bytes_per_step": int(o_host.numel() * 2)},
         "gpu_launches": args.steps * (1 if m <= PERSISTENT_MAX_M else 4 * shape.layers * 2),
+        "gemv": gemv,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -25,7 +25,10 @@ OPS = ("q", "k", "v", "o", "gate", "up", "down")
 EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv", "tq_gemm_workspace", "tq_gemm",
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
            "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
-           "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode", "tq_ldlq_workspace", "tq_ldlq_encode")
+           "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode", "tq_ldlq_workspace", "tq_ldlq_encode",
+           "tq_layer_stack_ex", "tq_workspace_status")
+TQ_STATUS_OFFSET = 65532
+TQ_GEMV_MAX_K = 53760
 
 
 class TqError(RuntimeError):
@@ -51,6 +54,10 @@ class tq_pack_info_t(ctypes.Structure):
 
 class tq_layer_t(ctypes.Structure):
     _fields_ = [(op, tq_weight_t) for op in OPS]
+
+
+class tq_stack_options_t(ctypes.Structure):
+    _fields_ = [("spin_limit", ctypes.c_uint32), ("test_skip_arrive", ctypes.c_int32)]
 
 
 _L = None
@@ -81,6 +88,9 @@ def _lib():
             "tq_layer_stack_workspace": ([LY, i32, i32, szp], ctypes.c_int),
             "tq_layer_phase": ([LY, i32, vp, i32, u64, vp, vp, vp, sz, vp], ctypes.c_int),
             "tq_layer_stack": ([LY, i32, vp, i32, u64, vp, vp, sz, vp], ctypes.c_int),
+            "tq_layer_stack_ex": ([LY, i32, vp, i32, u64, vp, vp, sz, ctypes.POINTER(tq_stack_options_t), vp],
+                                  ctypes.c_int),
+            "tq_workspace_status": ([vp, ctypes.POINTER(ctypes.c_int32), vp], ctypes.c_int),
             "tq_layer_stack_buffers": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_layer_stack_outputs": ([LY, i32, i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
             "tq_encode": ([vp, i32, i32, vp, ctypes.c_float, i32, vp, vp, vp, vp], ctypes.c_int),
@@ -275,6 +285,24 @@ class StackArgs:
 def tq_layer_stack(args: StackArgs, h_in, seed: int, h_out, ws, stream=None):
     _ok(_lib().tq_layer_stack(args.arr, args.n_layers, _ptr(h_in), args.m, seed, _ptr(h_out), _ptr(ws), ws.numel(),
                               _stream(stream)), "tq_layer_stack")
+
+
+def tq_layer_stack_ex(args: StackArgs, h_in, seed: int, h_out, ws, spin_limit: int = 0, test_skip_arrive: int = -1,
+                      stream=None):
+    """tq_layer_stack with options: the bounded waits' poll limit (0 = the
+    default) and the timeout test hook (a thread block that skips its arrive
+    at the first grid barrier; -1 = off)."""
+    opt = tq_stack_options_t(spin_limit, test_skip_arrive)
+    _ok(_lib().tq_layer_stack_ex(args.arr, args.n_layers, _ptr(h_in), args.m, seed, _ptr(h_out), _ptr(ws),
+                                 ws.numel(), ctypes.byref(opt), _stream(stream)), "tq_layer_stack_ex")
+
+
+def tq_workspace_status(ws, stream=None) -> int:
+    """The workspace's device status word (TQ_OK or TQ_ERR_TIMEOUT) once the
+    stream has reached this call (synchronises the stream)."""
+    v = ctypes.c_int32()
+    _ok(_lib().tq_workspace_status(_ptr(ws), ctypes.byref(v), _stream(stream)), "tq_workspace_status")
+    return v.value
 
 
 def tq_encode(w_rot, codebook, gain: float, refits: int = 1, codes=None, scales=None, err=None, want_err=True,

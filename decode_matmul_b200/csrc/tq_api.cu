@@ -133,23 +133,30 @@ int dmma_lv_for(bool hilo, int32_t k) {
   return 0;
 }
 
+// Largest k of the batch-1 kernel: its 4 bytes of hi/lo activations per
+// feature sit in shared memory beside one 16 KB codebook copy (227 KB per
+// block), rounded down to a multiple of 512.
+constexpr int32_t kGemvMaxK = (int32_t)(((227 * 1024 - 16384) / 4) / 512 * 512);
+
 template <int LV, int NT, bool HILO>
-int dmma_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream) {
+int dmma_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream, bool dry_run) {
   auto kern = tq::dmma_kernel<LV, NT, HILO>;
   const size_t smem = (16384u << LV) + (HILO ? (size_t)p.k * 4 : 0);
+  if (smem > 227 * 1024) return TQ_ERR_SHAPE;
   // per instantiation and device: opt in to large shared memory once and
-  // remember the occupancy for each shared-memory size class seen
-  static int occ_cache[kMaxDevices][64];
+  // remember the occupancy for each shared-memory size (in KB) seen
+  static int occ_cache[kMaxDevices][228];
   int dev = 0;
   TQ_CUDA(cudaGetDevice(&dev));
-  const int cls = (int)(smem >> 12) & 63;
+  const int cls = (int)((smem + 1023) >> 10);
   int occ = occ_cache[dev][cls];
   if (occ == 0) {
     TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-    TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, smem));
+    TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA_THREADS, cls << 10));
     if (occ < 1) return TQ_ERR_SHAPE;
     occ_cache[dev][cls] = occ;
   }
+  if (dry_run) return TQ_OK;
   int64_t grid = (int64_t)num_sms * occ;
   const int64_t need = (p.units + tq::DMMA_WARPS - 1) / tq::DMMA_WARPS;
   if (grid > need) grid = need;
@@ -161,19 +168,23 @@ int dmma_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream) {
 }
 
 template <int NT, bool HILO>
-int dmma_launch_lv(DmmaParams& p, int lv, int num_sms, cudaStream_t stream) {
+int dmma_launch_lv(DmmaParams& p, int lv, int num_sms, cudaStream_t stream, bool dry_run) {
   switch (lv) {
-    case 3: return dmma_launch_t<3, NT, HILO>(p, num_sms, stream);
-    case 2: return dmma_launch_t<2, NT, HILO>(p, num_sms, stream);
-    case 1: return dmma_launch_t<1, NT, HILO>(p, num_sms, stream);
-    default: return dmma_launch_t<0, NT, HILO>(p, num_sms, stream);
+    case 3: return dmma_launch_t<3, NT, HILO>(p, num_sms, stream, dry_run);
+    case 2: return dmma_launch_t<2, NT, HILO>(p, num_sms, stream, dry_run);
+    case 1: return dmma_launch_t<1, NT, HILO>(p, num_sms, stream, dry_run);
+    default: return dmma_launch_t<0, NT, HILO>(p, num_sms, stream, dry_run);
   }
 }
 
-// Fill the shape / workspace fields of p and launch.  p.m <= 32.
-int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream) {
+// Fill the shape / workspace fields of p and launch.  p.m <= 32.  With
+// dry_run every check (shape, workspace, shared-memory fit, occupancy) runs
+// and nothing is launched.
+int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream,
+             bool dry_run = false) {
   const int nt = hilo ? 1 : dmma_nt_for(p.m);
   const int mc = hilo ? 1 : nt * 8;
+  if (hilo && p.k > kGemvMaxK) return TQ_ERR_SHAPE;
   const DmmaWs L = dmma_ws_layout(p.n_total, p.k, mc);
   if (!ws) return TQ_ERR_WORKSPACE;
   if (ws_bytes < L.bytes) return TQ_ERR_WORKSPACE;
@@ -185,11 +196,11 @@ int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, c
   p.counters = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.counters_off);
   p.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + L.partials_off);
   const int lv = dmma_lv_for(hilo, p.k);
-  if (hilo) return dmma_launch_lv<1, true>(p, lv, num_sms, stream);
+  if (hilo) return dmma_launch_lv<1, true>(p, lv, num_sms, stream, dry_run);
   switch (nt) {
-    case 1: return dmma_launch_lv<1, false>(p, lv, num_sms, stream);
-    case 2: return dmma_launch_lv<2, false>(p, lv, num_sms, stream);
-    default: return dmma_launch_lv<4, false>(p, lv, num_sms, stream);
+    case 1: return dmma_launch_lv<1, false>(p, lv, num_sms, stream, dry_run);
+    case 2: return dmma_launch_lv<2, false>(p, lv, num_sms, stream, dry_run);
+    default: return dmma_launch_lv<4, false>(p, lv, num_sms, stream, dry_run);
   }
 }
 
@@ -210,6 +221,7 @@ void dmma_single(DmmaParams& p, const tq_weight_t* w) {
 constexpr int kUmmaMinM = 32;  // from this many tokens on the decoded GEMM uses tcgen05 (measured crossover)
 constexpr int kSplitTarget = 148;    // split k until about one CTA per SM (B200 SM count)
 constexpr int kStatusOff = (int)kCounterBytes - 4;  // error word: last 4 bytes of the counter region
+static_assert(kStatusOff == TQ_STATUS_OFFSET, "the status word offset is part of the interface");
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
@@ -520,6 +532,7 @@ int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* worksp
             void* stream) {
   int st = check_weight(w);
   if (st != TQ_OK) return st;
+  if (w->k > kGemvMaxK) return TQ_ERR_SHAPE;
   if (!x_rot_d || !y_d) return TQ_ERR_NULL;
   if (!aligned16(x_rot_d) || !aligned16(y_d)) return TQ_ERR_ALIGN;
   int sms = 0;
@@ -581,6 +594,17 @@ int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float*
     st = dmma_run(p, false, workspace_d, ws_bytes, sms, (cudaStream_t)stream);
     if (st != TQ_OK) return st;
   }
+  return TQ_OK;
+}
+
+int tq_workspace_status(const void* workspace_d, int32_t* status, void* stream) {
+  if (!workspace_d || !status) return TQ_ERR_NULL;
+  int32_t v = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  TQ_CUDA(cudaMemcpyAsync(&v, static_cast<const char*>(workspace_d) + TQ_STATUS_OFFSET, sizeof(v),
+                          cudaMemcpyDeviceToHost, s));
+  TQ_CUDA(cudaStreamSynchronize(s));
+  *status = v;
   return TQ_OK;
 }
 
@@ -715,7 +739,8 @@ static size_t stack_y_offset(const StackWs& L, int32_t m, int phase) {
 // nothing) when the stack does not qualify: more than STACK_MAX_LAYERS layers,
 // phases with different codebooks, or a phase too wide for shared memory.
 static int stack_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in, int32_t m, uint64_t seed,
-                     uint16_t* h_out, char* ws, const StackWs& L, int sms, cudaStream_t s) {
+                     uint16_t* h_out, char* ws, const StackWs& L, int sms, const tq_stack_options_t* opt,
+                     cudaStream_t s) {
   if (n_layers > tq::STACK_MAX_LAYERS || sms > kStackMaxCtas) return TQ_ERR_SHAPE;
   static thread_local tq::StackParams sp;  // large (~25 KB): per-thread storage, copied into the launch
   memset(&sp, 0, sizeof(sp));
@@ -771,7 +796,8 @@ static int stack_run(const tq_layer_t* layers, int32_t n_layers, const uint16_t*
   sp.partials = reinterpret_cast<float*>(ws + kCounterBytes);
   sp.sync = reinterpret_cast<uint32_t*>(ws + L.sync);
   sp.phase_table = reinterpret_cast<uint4*>(ws + L.params);
-  sp.spin_limit = 1u << 24;  // x 64 ns sleeps: ~1 s, far above any healthy phase
+  sp.spin_limit = (opt && opt->spin_limit) ? opt->spin_limit : (1u << 24);  // x 64 ns sleeps: ~1 s by default
+  sp.skip_arrive_cta = opt ? opt->test_skip_arrive : -1;
   void (*kern)(tq::StackParams);
   if (m > 1) {
     kern = nt == 1 ? tq::stackn_kernel<3, 1> : tq::stackn_kernel<3, 2>;
@@ -839,6 +865,14 @@ int tq_layer_stack_workspace(const tq_layer_t* layers, int32_t n_layers, int32_t
 
 int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m, uint64_t seed,
                    uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes, void* stream) {
+  return tq_layer_stack_ex(layers, n_layers, h_in_bf16_d, m, seed, h_out_bf16_d, workspace_d, ws_bytes, nullptr,
+                           stream);
+}
+
+int tq_layer_stack_ex(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m,
+                      uint64_t seed, uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes,
+                      const tq_stack_options_t* options, void* stream) {
+  if (options && options->test_skip_arrive < -1) return TQ_ERR_VALUE;
   if (m == 0) return TQ_OK;
   StackWs L;
   int st = stack_layout(layers, n_layers, m, &L);
@@ -857,7 +891,7 @@ int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h
   const size_t phase_bytes = L.y;
   cudaStream_t s = (cudaStream_t)stream;
   if (m <= kStackMaxM) {
-    st = stack_run(layers, n_layers, h_in_bf16_d, m, seed, h_out_bf16_d, ws, L, sms, s);
+    st = stack_run(layers, n_layers, h_in_bf16_d, m, seed, h_out_bf16_d, ws, L, sms, options, s);
     if (st != TQ_ERR_SHAPE) return st;  // TQ_ERR_SHAPE: not eligible, run phase by phase
   }
   for (int l = 0; l < n_layers; ++l) {
@@ -888,6 +922,7 @@ static_assert(TQ_GEMV_NOALLOC_SCRATCH_BYTES >= kCounterBytes + (size_t)tq::DMMA_
 int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* stream) {
   int st = check_weight(w);
   if (st != TQ_OK) return st;
+  if (w->k > kGemvMaxK) return TQ_ERR_SHAPE;
   if (!x_rot_d || !y_d) return TQ_ERR_NULL;
   if (!aligned16(x_rot_d) || !aligned16(y_d)) return TQ_ERR_ALIGN;
   if ((int64_t)(w->n + 15) / 16 > kMaxTiles || dmma_ws_layout(w->n, w->k, 1).bytes > TQ_GEMV_NOALLOC_SCRATCH_BYTES)
@@ -904,13 +939,17 @@ int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void
   }
   void* ws = g_gemv_scratch_addr[dev];
   cudaStream_t s = (cudaStream_t)stream;
-  // the arrival counters must start at zero whatever an earlier call left
-  TQ_CUDA(cudaMemsetAsync(ws, 0, kCounterBytes, s));
   DmmaParams p;
   dmma_single(p, w);
   p.m = 1;
   p.x_f32 = x_rot_d;
   p.y = y_d;
+  // every check first (nothing is enqueued on an error) ...
+  st = dmma_run(p, true, ws, TQ_GEMV_NOALLOC_SCRATCH_BYTES, sms, s, /*dry_run=*/true);
+  if (st != TQ_OK) return st;
+  // ... then the arrival counters, which must start at zero whatever an
+  // earlier call left, and the launch
+  TQ_CUDA(cudaMemsetAsync(ws, 0, kCounterBytes, s));
   return dmma_run(p, true, ws, TQ_GEMV_NOALLOC_SCRATCH_BYTES, sms, s);
 }
 

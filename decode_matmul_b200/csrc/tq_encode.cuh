@@ -284,8 +284,8 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(EncArgs a) {
 }
 
 // ---- block LDLQ feedback --------------------------------------------------------
-// "Pingala-8" landing page, "How it works": LDLQ rounding passes each column's
-// error on to the columns not yet coded.  With the proxy Hessian factored as
+// LDLQ, named on the "Pingala-8" landing page ("How it works"): the coding
+// error of the columns already coded is fed forward.  With the proxy Hessian factored as
 // H = (I + U) D (I + U)^T (U strictly upper by 256-column blocks), block b of
 // each row is encoded from
 //   wt[r][j] = w[r][256b + j] + sum_{i < 256b} delta[r][i] * U[i][256b + j],

@@ -65,6 +65,7 @@ struct StackParams {
   uint4* phase_table;     // [4 * n_layers][PARAM_QUADS]: every phase's parameters
   int32_t* status;
   uint32_t spin_limit;
+  int32_t skip_arrive_cta;  // test hook: this CTA does not arrive at the launch's first barrier (-1: none)
 };
 
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
@@ -112,9 +113,11 @@ __device__ __forceinline__ void stack_phase_params(const StackParams& sp, int f,
 }
 
 // Arrive at the grid barrier (after the whole CTA finished its writes).
-__device__ __forceinline__ void grid_arrive(const StackParams& sp) {
+// With arrive = false the CTA only synchronises itself (the test hook that
+// makes every bounded wait of the barrier run out).
+__device__ __forceinline__ void grid_arrive(const StackParams& sp, bool arrive = true) {
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && arrive) {
     __threadfence();
     atomicAdd(sp.sync, 1u);
   }
@@ -437,7 +440,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stack1_kernel(const __grid_co
     for (int i = 0; i < 32; ++i) bits |= (rht_sign_negative(seed_lp, k0 + i) ? 1u : 0u) << i;
     sp.signs[j] = bits;
   }
-  grid_arrive(sp);  // its __syncthreads publishes slots 0 and 1 to the CTA
+  grid_arrive(sp, (int)blockIdx.x != sp.skip_arrive_cta);  // its __syncthreads publishes slots 0 and 1
   uint32_t epoch = 1;
 
   // first phase's tables and code chunk, then the barrier

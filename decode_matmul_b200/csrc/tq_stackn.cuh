@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) stackn_kernel(const __grid_co
     for (int i = 0; i < 32; ++i) bits |= (rht_sign_negative(seed_lp, k0 + i) ? 1u : 0u) << i;
     sp.signs[j] = bits;
   }
-  grid_arrive(sp);  // its __syncthreads publishes slots 0 and 1 to the CTA
+  grid_arrive(sp, (int)blockIdx.x != sp.skip_arrive_cta);  // its __syncthreads publishes slots 0 and 1
   uint32_t epoch = 1;
   stack_warp_tables(slot(0), wbeg(0), wfirst(0), tid);
   if (!grid_wait(sp, epoch * gridDim.x, abort_flag)) return;

@@ -34,7 +34,8 @@
  *     Host pointers (structs, `out` arguments) are read or written before the
  *     call returns.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
- *     are asynchronous on it; none synchronises.
+ *     are asynchronous on it; none synchronises, except tq_workspace_status,
+ *     which reads a word of device memory back to the host.
  *   - Return value: TQ_OK or one TQ_ERR_* code.  On an error nothing is
  *     launched.  No C++ exception crosses this interface.
  *   - k must be a positive multiple of 512.  n >= 1.  m >= 0 (m == 0 and
@@ -134,7 +135,10 @@ TQ_API int tq_gemv_workspace(int32_t n, int32_t k, size_t* bytes);
  * before the first call (tq_workspace_init); every call of this library leaves
  * it zero again, so one workspace may serve calls of any shape in turn.  The
  * rest is scratch.  Calls that share a workspace must not overlap on the GPU.
- * n is limited to 262128 rows per call (TQ_ERR_SHAPE). */
+ * n is limited to 262128 rows per call and k to TQ_GEMV_MAX_K (the kernel
+ * keeps 4 bytes of activations per feature in shared memory beside a 16 KB
+ * codebook copy); beyond either, TQ_ERR_SHAPE before anything is launched. */
+#define TQ_GEMV_MAX_K 53760
 TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* workspace_d, size_t ws_bytes,
             void* stream);
 
@@ -154,8 +158,10 @@ TQ_API int tq_gemv(const tq_weight_t* w, const float* x_rot_d, float* y_d, void*
  * the array, which keeps the last call's contents: calls that overlap on the
  * GPU (for example on two streams) race and give wrong results, so run them
  * one after another.
- * Limit: n <= 262128 rows (TQ_ERR_SCRATCH beyond it); k any positive
- * multiple of 512. */
+ * Limits: n <= 262128 rows (TQ_ERR_SCRATCH beyond it); k a positive
+ * multiple of 512 up to TQ_GEMV_MAX_K (TQ_ERR_SHAPE beyond it).  Every check
+ * runs before the counter clear is enqueued: on an error nothing is
+ * enqueued. */
 #define TQ_GEMV_NOALLOC_SCRATCH_BYTES ((size_t)(1u << 20) + (size_t)(64u << 10))
 TQ_API int tq_gemv_noalloc(const tq_weight_t* w, const float* x_rot_d, float* y_d, void* stream);
 
@@ -173,6 +179,26 @@ TQ_API int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m,
 
 /* Zero a workspace (cudaMemsetAsync on `stream`). */
 TQ_API int tq_workspace_init(void* workspace_d, size_t bytes, void* stream);
+
+/* ---- device-side status ------------------------------------------------------
+ * Kernels that wait on other thread blocks (the tcgen05 GEMM's pipeline
+ * barriers, the persistent stack kernels' grid barriers and block flags) bound
+ * every wait.  When a wait runs out, the kernel writes TQ_ERR_TIMEOUT into the
+ * 32-bit status word at byte TQ_STATUS_OFFSET of the workspace it was given
+ * (the last word of the 64 KB counter region), stops and returns; its outputs
+ * are then undefined.  The host calls return before the kernels run, so they
+ * cannot report it: read the word after the stream has reached the call.
+ * No call of this library clears it except tq_workspace_init, and after a
+ * timeout the counter region may hold non-zero counts, so re-initialise the
+ * workspace (tq_workspace_init) before using it again.
+ * The batch-1 GEMV (tq_gemv, tq_gemv_noalloc) has no device-side wait (its
+ * split tiles are summed by the last block to arrive), so it never sets it. */
+#define TQ_STATUS_OFFSET 65532
+
+/* Copy the status word of `workspace_d` to *status (TQ_OK or TQ_ERR_TIMEOUT)
+ * after everything enqueued on `stream` before it.  The one call of this
+ * library that synchronises: it waits for `stream`.  Does not clear the word. */
+TQ_API int tq_workspace_status(const void* workspace_d, int32_t* status, void* stream);
 
 /* ---- layer stack ----------------------------------------------------------
  * One layer = q, k, v, o, gate, up, down.  Per layer, four phases run in
@@ -214,9 +240,38 @@ TQ_API int tq_layer_phase(const tq_layer_t* layer, int32_t phase, const uint16_t
 /* The whole stack: h_out = layers[n-1] o ... o layers[0] (h_in).
  * layers: HOST array of n_layers tq_layer_t (device pointers inside).
  * h_in_bf16_d / h_out_bf16_d: device bf16 [m][hidden]; they may alias.
- * Enqueues 4 phases per layer on `stream` (capturable in a CUDA graph). */
+ * For 1 <= m <= 16 every phase of every layer runs in ONE cooperative
+ * persistent launch: one thread block per SM, all of them resident at once,
+ * with bounded grid-wide waits between phases (the launch fails with
+ * TQ_ERR_CUDA when the blocks cannot all be resident, e.g. when other work
+ * holds SMs; a wait that runs out leaves TQ_ERR_TIMEOUT in the status word).
+ * A stack that does not fit that kernel (more than 128 layers, phases with
+ * different codebooks, a phase too wide for shared memory) and m > 16 run as
+ * 4 launch groups per layer (RHT + matmul), PDL-chained on `stream`.  Either
+ * way the work is enqueued on `stream` and can be captured in a CUDA graph. */
 TQ_API int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m, uint64_t seed,
                    uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes, void* stream);
+
+/* Options of tq_layer_stack_ex.
+ * spin_limit: polls each bounded wait of the persistent kernels makes before
+ *   it gives up (each poll is one L2 round trip plus a 64 ns sleep); 0 = the
+ *   default, about a second, far above any healthy wait.
+ * test_skip_arrive: a fault-injection hook for tests of the timeout path.
+ *   -1 = off.  c >= 0: thread block c of the persistent kernel does not
+ *   arrive at the launch's first grid barrier, so every block's bounded wait
+ *   there runs out; the launch ends early with TQ_ERR_TIMEOUT in the status
+ *   word and undefined outputs.  Values below -1 are TQ_ERR_VALUE; a block
+ *   index past the grid makes nothing happen.  Ignored by the per-phase path
+ *   (m > 16). */
+typedef struct tq_stack_options {
+  uint32_t spin_limit;
+  int32_t test_skip_arrive;
+} tq_stack_options_t;
+
+/* tq_layer_stack with options (NULL = the defaults, which is tq_layer_stack). */
+TQ_API int tq_layer_stack_ex(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m,
+                             uint64_t seed, uint16_t* h_out_bf16_d, void* workspace_d, size_t ws_bytes,
+                             const tq_stack_options_t* options, void* stream);
 
 /* Byte offsets, inside a tq_layer_stack workspace for these layers and m,
  * of the bf16 buffers that hold the last layer's phase handoffs when
@@ -274,9 +329,9 @@ TQ_API int tq_layer_stack_outputs(const tq_layer_t* layers, int32_t n_layers, in
 TQ_API int tq_encode(const float* w_rot_d, int32_t n, int32_t k, const uint16_t* codebook_d, float gain, int32_t refits,
                      uint8_t* codes_d, uint16_t* scales_d, float* err_d, void* stream);
 
-/* Block LDLQ with the trellis encoder ("Pingala-8" landing page, "How it
- * works": LDLQ rounding passes each column's error on to the columns not yet
- * coded).  The proxy Hessian of the layer's inputs is given by its factor:
+/* Block LDLQ with the trellis encoder (the LDLQ step named on the
+ * "Pingala-8" landing page, section "How it works"; the feedback it applies
+ * is the equation below).  The proxy Hessian of the layer's inputs is given by its factor:
  * H = (I + U) D (I + U)^T with U strictly upper triangular by 256-column
  * blocks (U[i][j] = 0 unless i/256 < j/256; D, block diagonal, is not needed).
  * For each 256-column block b in order, every row is encoded (as tq_encode)

@@ -497,8 +497,8 @@ void orc_encode32(const float* w, int64_t n, int64_t k, const uint16_t* cb, floa
 /* ======================================================================== */
 /* Block LDLQ with the trellis encoder.                                      */
 /*                                                                           */
-/* "Pingala-8" landing page, "How it works": LDLQ rounding passes each       */
-/* column's error on to the columns not yet coded.  Reading adopted: with    */
+/* LDLQ, named on the "Pingala-8" landing page ("How it works"): the coding */
+/* error of the columns already coded is fed forward.  Reading adopted: with */
 /* the proxy Hessian factored as H = (I + U) D (I + U)^T, U strictly upper   */
 /* triangular by 256-column blocks, block b of each row is encoded from       */
 /*   w~_b = w_b + (w - w_hat)_{<b} U_{<b,b}                                  */

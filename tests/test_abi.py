@@ -109,6 +109,25 @@ def test_argument_checks_before_any_device_call():
     assert L.tq_gemm(ctypes.byref(W), 16, 0, 16, 16, 1 << 20, None) == tq.TQ_OK
 
 
+def test_gemv_k_limit_and_new_entry_points_checks():
+    L = tq.lib()
+    past = tq.tq_weight_t(16, 16, 16, 32, tq.TQ_GEMV_MAX_K + 512)
+    # one 512-block past the batch-1 shared-memory limit: refused before any device call
+    assert L.tq_gemv(ctypes.byref(past), 16, 16, 16, 1 << 30, None) == tq.TQ_ERR_SHAPE
+    assert L.tq_gemv_noalloc(ctypes.byref(past), 16, 16, None) == tq.TQ_ERR_SHAPE
+    assert tq.TQ_GEMV_MAX_K % 512 == 0 and 16384 + 4 * tq.TQ_GEMV_MAX_K <= 227 * 1024
+    assert 16384 + 4 * (tq.TQ_GEMV_MAX_K + 512) > 227 * 1024
+    # status query
+    v = ctypes.c_int32()
+    assert L.tq_workspace_status(None, ctypes.byref(v), None) == tq.TQ_ERR_NULL
+    assert L.tq_workspace_status(16, None, None) == tq.TQ_ERR_NULL
+    # stack options: a negative block index other than -1 is refused first
+    layers = [_fake_layer(1024, 1536, 256, 2560)]
+    arr = (tq.tq_layer_t * 1)(*layers)
+    opt = tq.tq_stack_options_t(0, -2)
+    assert L.tq_layer_stack_ex(arr, 1, 16, 1, 0, 16, 16, 1 << 30, ctypes.byref(opt), None) == tq.TQ_ERR_VALUE
+
+
 def test_stack_phase_seed_matches_oracle():
     # both sides implement SplitMix64 from its published definition
     for s, l, p in [(0, 0, 0), (0, 35, 3), (12345, 7, 2), (2 ** 64 - 1, 63, 1)]:

@@ -46,3 +46,32 @@ def test_clock_summary_keeps_the_timed_region_only():
                 "0, 1900, 1965, 710.0, 0x4, Not Active, Not Active, Not Active, Active"]
     s2 = c2.summary()
     assert s2["samples"] == 2 and s2["reasons"] == ["sw_power_cap"] and s2["source"] == "nvidia-smi"
+
+
+def test_oracle_baseline_uses_every_host_core_and_one():
+    sys.path.insert(0, ROOT)
+    import bench
+    import tqsynth
+    shape = tqsynth.StackShape("tiny", 2, 512, 512, 512, 1024)
+    d = bench.oracle_baseline(shape, 1, budget_s=0.3)
+    assert d["kind"] == "oracle" and d["unit"] == "tok/s"
+    assert d["cores"] == bench.host_cores() >= 1
+    assert d["value"] > 0 and d["single_thread_value"] > 0
+    assert "phase seeds" in d["sample"]
+
+
+def test_ncu_traffic_only_for_the_kernel_it_was_taken_on(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (tmp_path / "decode_matmul_b200").symlink_to(os.path.join(ROOT, "decode_matmul_b200"))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"workload": "qwen3-4b-shaped", "dram_bytes_per_layer": 1000.0, "source_sha256": bench.kernel_source_hash()}
+    (prof / "stack1_kernel_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("qwen3-4b-shaped", 36, 1) == 36000.0
+    assert bench.ncu_traffic("qwen3-4b-shaped", 36, 2) is None
+    assert bench.ncu_traffic("27b-class", 64, 1) is None
+    rec["source_sha256"] = "0" * 64
+    (prof / "stack1_kernel_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("qwen3-4b-shaped", 36, 1) is None

@@ -1,6 +1,7 @@
 """The CUDA path at the documented size limits, against the oracle on sampled
-outputs: the most rows a decode-GEMV call takes (262128 = 16383 tiles of 16)
-and the most tokens a GEMM call takes (4096); one past each is rejected."""
+outputs: the most rows a decode-GEMV call takes (262128 = 16383 tiles of 16),
+the widest input it takes (TQ_GEMV_MAX_K = 53760 features) and the most
+tokens a GEMM call takes (4096); one past each is rejected."""
 import ctypes
 
 import numpy as np
@@ -55,3 +56,25 @@ def test_gemm_at_the_token_limit():
     with pytest.raises(tq.TqError) as e:
         tq.tq_gemm_workspace(n, k, m + 1)
     assert e.value.status == tq.TQ_ERR_SHAPE
+
+
+def test_gemv_at_the_k_limit():
+    import torch
+
+    import decode_matmul_b200 as tq
+    n, k = 40, tq.TQ_GEMV_MAX_K
+    hw = host_weight(5, 0, 4, n, k)
+    x = tqsynth.activations(5, 1, k)
+    xr = f32_exact(oracle.rht(x, 1, k, 23))
+    dw = dev_weight(hw)
+    xd = torch.from_numpy(xr.astype(np.float32)).cuda()
+    y = tq.tq_gemv(dw, xd).cpu().numpy()
+    want = oracle.linear(hw.codes, hw.scales, hw.codebook, n, k, xr, 1)[0]
+    assert oracle.rel_err(y, want) < 1e-4
+    # one 512-block wider does not fit shared memory: refused, nothing launched
+    wide = tq.tq_weight_t(dw.codes.data_ptr(), dw.scales.data_ptr(), dw.codebook.data_ptr(), n, k + 512)
+    ws = tq.workspace(tq.tq_gemv_workspace(n, k + 512))
+    yb = torch.empty(n, dtype=torch.float32, device="cuda")
+    st = tq.lib().tq_gemv(ctypes.byref(wide), ctypes.c_void_p(xd.data_ptr()), ctypes.c_void_p(yb.data_ptr()),
+                          ctypes.c_void_p(ws.data_ptr()), ws.numel(), None)
+    assert st == tq.TQ_ERR_SHAPE

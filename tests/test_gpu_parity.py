@@ -39,6 +39,20 @@ def test_decode_bit_exact(tq, torch_cuda, n, k):
     assert np.array_equal(got, want)
 
 
+
+@pytest.mark.parametrize("n,k", [(2560, 9728), (4096, 14336), (5120, 17408)])
+def test_decode_bit_exact_down_projection_widths(tq, torch_cuda, n, k):
+    # the down projections of the three stacks (Qwen3-4B, Llama-3.1-8B and
+    # 27B-class shapes), decoded whole on the GPU; sampled rows (first, last,
+    # a tile boundary and 60 seeded others) against the oracle bit for bit
+    hw = host_weight(0, 1, 6, n, k)
+    got = from_dev_u16(tq.tq_decode(dev_weight(hw)))
+    assert got.shape == (n, k)
+    rows = sorted({0, 1, 15, 16, n // 2, n - 2, n - 1} | set(np.random.default_rng(k).integers(0, n, 60).tolist()))
+    for r in rows:
+        want = oracle.decode_rows(hw.codes, hw.scales, hw.codebook, k, r, r + 1)[0]
+        assert np.array_equal(got[r], want), r
+
 def test_decode_hand_codebook_block_reset(tq, torch_cuda):
     # the hand-worked example of tests/golden (block reset at group 64)
     s = np.arange(8)[:, None, None]
