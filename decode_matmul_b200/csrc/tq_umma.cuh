@@ -14,9 +14,21 @@
 //   warp 1      TMEM allocation; one thread issues tcgen05.mma (M=128,
 //               N=BN, K=16, fp16 x fp16 -> fp32) and tcgen05.commit
 //   warps 4-11  decoders: two threads per row, 8 codes each (codebook in
-//               shared memory, exact fp16 scale * entry), into the K-major
-//               128B-swizzled A tile; then the epilogue (tcgen05.ld), warps
-//               4-7 and 8-11 taking one half of the columns each
+//               shared memory, exact fp16 scale * entry), into the MMA's A
+//               operand; then the epilogue (tcgen05.ld), warps 4-7 and 8-11
+//               taking one half of the columns each
+// Where A lives depends on the tile width:
+//   * up to 128 tokens, in shared memory (the K-major 128B-swizzled tile);
+//     at 64 tokens the stage ring is 6 deep, which measured 15% faster than
+//     4 on the 27B-class gate|up shape at 32 tokens: the loop is bound by
+//     the latency of the stage round trip (TMA in, decode, MMA, release),
+//     not by shared-memory bandwidth;
+//   * at 256 tokens, in tensor memory (tcgen05.st by the decoders; row r of
+//     the tile in TMEM lane r, the fp16 pair (2c, 2c+1) of the k step in
+//     column c of the stage), because there the loop is bound by shared
+//     memory and a decoded tile in shared memory costs a 16 KB write and a
+//     16 KB MMA read per k step (9% faster on the Qwen3-4B gate|up shape at
+//     512 tokens).
 // Stages are handed over with mbarriers; every wait is bounded and, when it
 // runs out, the kernel records TQ_ERR_TIMEOUT in the status word and drains.
 #pragma once
@@ -113,6 +125,30 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b
       : "memory");
 }
 
+// The same MMA with A read from tensor memory (tmem_a: lane = row, 32-bit
+// column = two consecutive k).
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                                uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (warp-collective:
+// lanes 32 (warp % 4) .. + 31).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
                : "memory");
@@ -143,12 +179,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 template <int BN>
 struct UmmaSmem {
-  // 4 stages; the codebook as 4 views (64 KB) where that still fits (64 and
-  // 128 tokens), a single copy at 256 tokens (3 stages + 4 views measured
-  // slower there than 4 stages + one copy)
-  static constexpr int STAGES = 4;
-  static constexpr int LV = BN == 256 ? 0 : 2;
-  static constexpr uint32_t A_BYTES = UM_BM * 128;     // 16 KB per stage
+  // A in tensor memory at 256 tokens (see the file header)
+  static constexpr bool TMEM_A = BN == 256;
+  // stages: 6 at 64 tokens, 4 above; the codebook as 4 views (64 KB)
+  static constexpr int STAGES = BN == 64 ? 6 : 4;
+  static constexpr int LV = 2;
+  // TMEM columns: the fp32 accumulator [0, BN), then (TMEM_A) 32 per stage
+  static constexpr uint32_t A_COL0 = BN;
+  static constexpr uint32_t TMEM_COLS = TMEM_A ? 512 : BN;
+  static constexpr uint32_t A_BYTES = TMEM_A ? 0 : UM_BM * 128;  // 16 KB per stage in shared memory
   static constexpr uint32_t B_BYTES = BN * 128;        // BN rows of 64 fp16
   static constexpr uint32_t C_BYTES = UM_BM * 16;      // 16 code bytes per row
   static constexpr uint32_t A_OFF = 0;
@@ -159,6 +198,8 @@ struct UmmaSmem {
   static constexpr uint32_t MISC_OFF = BAR_OFF + (3 * STAGES + 1) * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 64;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // slack to align the base to 1024
+  static_assert(ALLOC <= 227 * 1024, "shared memory per block");
+  static_assert(!TMEM_A || A_COL0 + 32 * STAGES <= TMEM_COLS, "tensor memory columns");
 };
 
 template <int BN>
@@ -220,7 +261,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
-                 "r"(BN));
+                 "r"(L::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
   tc_fence_before();
@@ -266,11 +307,19 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = base + L::A_OFF + s * L::A_BYTES, b0 = base + L::B_OFF + s * L::B_BYTES;
+        const uint32_t b0 = base + L::B_OFF + s * L::B_BYTES;
+        if (L::TMEM_A) {
+          const uint32_t a0 = tmem + L::A_COL0 + s * 32;
 #pragma unroll
-        for (int k16 = 0; k16 < UM_BK / 16; ++k16)
-          umma_f16(tmem, umma_smem_desc(a0 + k16 * 32), umma_smem_desc(b0 + k16 * 32), idesc,
-                   (i > 0 || k16 > 0) ? 1u : 0u);
+          for (int k16 = 0; k16 < UM_BK / 16; ++k16)
+            umma_f16_tmem_a(tmem, a0 + k16 * 8, umma_smem_desc(b0 + k16 * 32), idesc, (i > 0 || k16 > 0) ? 1u : 0u);
+        } else {
+          const uint32_t a0 = base + L::A_OFF + s * L::A_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < UM_BK / 16; ++k16)
+            umma_f16(tmem, umma_smem_desc(a0 + k16 * 32), umma_smem_desc(b0 + k16 * 32), idesc,
+                     (i > 0 || k16 > 0) ? 1u : 0u);
+        }
         umma_commit(bar_empty + 8 * s);
       }
       umma_commit(bar_acc);  // arrives once every MMA issued above has completed
@@ -280,6 +329,9 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     const int dt = tid - 128;
     const int r = dt & (UM_BM - 1);  // row of the tile
     const int h = dt >> 7;           // codes 8h .. 8h+7 of each 16-code chunk
+    // (TMEM_A) this thread's TMEM lane (row r: warps 4-7 and 8-11 hold rows
+    // 32 (warp % 4) ..) and its 16 columns (codes 8h .. 8h+7) of a stage
+    const uint32_t a_thr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + L::A_COL0 + 16 * h;
     const int grow = min(row0 + r, p.n_total - 1);
     const uint16_t* srow = p.scales[seg] + (size_t)(grow - p.seg_row0[seg]) * blocks;
     const uint8_t* cbs = sm + L::CB_OFF + ((lane & ((1 << L::LV) - 1)) << 3);
@@ -303,23 +355,29 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
       const uint32_t w0 = h ? cw.z : cw.x, w1 = h ? cw.w : cw.y;
       uint32_t prev = h ? (cw.y >> 24) : carry;
       carry = cw.w >> 24;
-      uint8_t* arow = sm + L::A_OFF + s * L::A_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+      uint32_t out[16];  // 4-byte words 2j, 2j + 1: weights (0, 1), (2, 3) of code 8h + j
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {  // chunk 4h + c = codes 8h+2c, 8h+2c+1
-        uint32_t out[4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int j = 2 * c + hh;
-          const uint32_t code = ((j < 4 ? w0 : w1) >> (8 * (j & 3))) & 0xFFu;
-          const uint32_t e = ((prev & 7u) << 8) | code;
-          const uint2 ent = *reinterpret_cast<const uint2*>(cbs + (e << (3 + L::LV)));
-          out[2 * hh] = hmul2_u32(ent.x, sc2);
-          out[2 * hh + 1] = hmul2_u32(ent.y, sc2);
-          prev = code;
-        }
-        *reinterpret_cast<uint4*>(arow + (((4 * h + c) ^ (r & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t code = ((j < 4 ? w0 : w1) >> (8 * (j & 3))) & 0xFFu;
+        const uint32_t e = ((prev & 7u) << 8) | code;
+        const uint2 ent = *reinterpret_cast<const uint2*>(cbs + (e << (3 + L::LV)));
+        out[2 * j] = hmul2_u32(ent.x, sc2);
+        out[2 * j + 1] = hmul2_u32(ent.y, sc2);
+        prev = code;
       }
-      fence_async_smem();
+      if (L::TMEM_A) {
+        tc_fence_after();  // the stage's previous MMAs (released through bar_full's producer wait) are done
+        tmem_st16(a_thr + s * 32, out);
+        tmem_wait_st();
+        tc_fence_before();
+      } else {
+        uint8_t* arow = sm + L::A_OFF + s * L::A_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)  // 16-byte chunk 4h + c = codes 8h+2c, 8h+2c+1
+          *reinterpret_cast<uint4*>(arow + (((4 * h + c) ^ (r & 7)) << 4)) =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        fence_async_smem();
+      }
       mbar_arrive(bar_dec + 8 * s);
     }
   }
@@ -427,7 +485,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(BN));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(L::TMEM_COLS));
   }
 }
 
