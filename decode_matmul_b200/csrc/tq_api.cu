@@ -395,9 +395,13 @@ size_t matmul_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
   return round_up(b, 256);
 }
 
+// Bytes of x' for m tokens of k features: fp16, whole groups of 8 tokens
+// (the small-batch kernel's fragment order, tq::xt_pos).
+size_t xt_bytes(int64_t m, int64_t k) { return round_up((size_t)((m + 7) / 8 * 8) * k * 2, 256); }
+
 size_t phase_ws_bytes(int64_t n_total, int32_t k, int32_t m) {
   size_t b = matmul_ws_bytes(n_total, k, m);
-  if (m > 1) b += round_up((size_t)m * k * 2, 256);
+  if (m > 1) b += xt_bytes(m, k);
   return b;
 }
 
@@ -550,7 +554,7 @@ int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes) {
   if (!bytes) return TQ_ERR_NULL;
   if (n < 1 || !k_ok(k) || m < 0 || m > 4096) return TQ_ERR_SHAPE;
   *bytes = matmul_ws_bytes(n, k, m < 1 ? 1 : m);
-  if (m > 1 && m < kUmmaMinM) *bytes += round_up((size_t)m * k * 2, 256);  // x' in fragment order
+  if (m > 1 && m < kUmmaMinM) *bytes += xt_bytes(m, k);  // x' in fragment order
   return TQ_OK;
 }
 
@@ -575,7 +579,7 @@ int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float*
   // the small-batch kernel reads x' in fragment order: permute it into the
   // workspace after the matmul scratch
   const size_t mm_bytes = matmul_ws_bytes(w->n, w->k, m);
-  if (ws_bytes < mm_bytes + (size_t)m * w->k * 2) return TQ_ERR_WORKSPACE;
+  if (ws_bytes < mm_bytes + xt_bytes(m, w->k)) return TQ_ERR_WORKSPACE;
   uint16_t* xp = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace_d) + mm_bytes);
   {
     const int64_t groups = (int64_t)m * (w->k / 4);
@@ -720,7 +724,7 @@ static int stack_layout(const tq_layer_t* layers, int32_t n_layers, int32_t m, S
   L->sign_words = (uint32_t)words;
   L->params = L->signs + round_up((size_t)words * 4, 256);
   L->xq = L->params + round_up((size_t)n_layers * 4 * tq::PARAM_QUADS * 16, 256);
-  L->sync = L->xq + (m > 1 && m <= kStackMaxM ? round_up((size_t)m * kmax * 2, 256) : 0);
+  L->sync = L->xq + (m > 1 && m <= kStackMaxM ? xt_bytes(m, kmax) : 0);
   L->total = L->sync + 256;
   return TQ_OK;
 }

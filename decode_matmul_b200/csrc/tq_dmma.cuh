@@ -55,7 +55,7 @@ struct DmmaParams {
   const float* x_f32;      // batch 1: x' fp32 [k]
   const uint16_t* x_bf16;  // batch 1, fused RHT: x bf16 [k]
   uint64_t rht_seed;
-  const uint16_t* x_f16;   // small batch: x' fp16 [m][k] in fragment order (frag_pos)
+  const uint16_t* x_f16;   // small batch: x' fp16 in fragment order (xt_pos), whole groups of 8 tokens
   float* y;                // [m][n_total] or null
   uint16_t* handoff;       // [m][handoff_rows] bf16 or null
   int32_t handoff_rows;
@@ -498,8 +498,9 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
     const uint16_t* xg_lane[NT];
     uint4 bpair[NT];
 #pragma unroll
-    for (int jt = 0; jt < NT; ++jt)
-      xg_lane[jt] = p.x_f16 + (size_t)min(jt * 8 + g, p.m - 1) * p.k + (size_t)b * 256 + q * 8;
+    for (int jt = 0; jt < NT; ++jt)  // step pair 0 of block b, tokens 8 jt .. 8 jt + 7 (xt_pos); column
+      // tiles past the last group of 8 tokens re-read it (their outputs are discarded)
+      xg_lane[jt] = p.x_f16 + (size_t)min(jt, (p.m - 1) >> 3) * 8 * p.k + (size_t)b * 2048 + lane * 8;
     // previous code byte of each row chunk (state of code 0); 0 at a block start
     uint32_t pa = __shfl_up_sync(0xffffffffu, cur.ca.w, 1) >> 24;
     uint32_t pb = __shfl_up_sync(0xffffffffu, cur.cb.w, 1) >> 24;
@@ -536,8 +537,8 @@ __device__ __forceinline__ void dmma_units(const DmmaParams& p, const uint8_t* s
           if ((j & 1) == 0) {
 #pragma unroll
             for (int jt = 0; jt < NT; ++jt)
-              bpair[jt] = XCG ? __ldca(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j))
-                              : __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 16 * j));
+              bpair[jt] = XCG ? __ldca(reinterpret_cast<const uint4*>(xg_lane[jt] + 128 * j))
+                              : __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 128 * j));
           }
 #pragma unroll
           for (int jt = 0; jt < NT; ++jt) {

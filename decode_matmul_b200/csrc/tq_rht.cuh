@@ -67,22 +67,27 @@ __device__ __forceinline__ void rht512_warp(const uint16_t* __restrict__ x_row, 
   for (int r = 0; r < 16; ++r) v[r] *= inv;
 }
 
-// Position of element k of a row in "fragment order": inside each 256-weight
-// block the 64 groups of 4 (group 16q + j is read by lanes with q = lane % 4
-// at MMA step j of the small-batch kernel) are stored as (j / 2, q, j % 2):
-// a lane's quads of steps j and j + 1 are one 16-byte load, and the four
-// lanes of a step pair read 64 contiguous bytes.
-__host__ __device__ __forceinline__ int frag_pos(int k) {
-  const int b = k >> 8, G = (k & 255) >> 2, e = k & 3;
+// Offset of element kk of token t in "fragment order", the small-batch
+// kernel's x' layout.  Tokens go in groups of 8 (group t / 8 takes 8 k
+// elements per feature); inside a group's 256-weight block b, the 64 groups
+// of 4 weights (group 16q + j is read by lanes with q = lane % 4 at MMA step
+// j) of token g = t % 8 are stored as [j / 2][g][q][j % 2]: a lane's quads of
+// steps j and j + 1 are one 16-byte load, and the 32 lanes (g, q) of a step
+// pair read 512 contiguous bytes (four shared-memory-sized wavefronts; with
+// one row per token they touched eight lines).  Buffers hold whole groups of
+// 8 tokens; the rows past m are never written and feed only MMA columns whose
+// outputs are discarded.
+__host__ __device__ __forceinline__ size_t xt_pos(int t, int kk, int k) {
+  const int b = kk >> 8, G = (kk & 255) >> 2, e = kk & 3;
   const int j = G & 15, q = G >> 4;
-  return (b << 8) + ((((j >> 1) << 3) + (q << 1) + (j & 1)) << 2) + e;
+  return (size_t)(t >> 3) * 8 * k + (size_t)((b << 3) + (j >> 1)) * 256 + ((t & 7) << 5) + (q << 3) + ((j & 1) << 2) + e;
 }
 
 // Standalone RHT.  CTA (blk, y) transforms 512-block `blk` of rows 8y + warp
 // (grid-stride in y): the 512 diagonal signs of the block are hashed once per
 // CTA (two per thread, packed by ballot into shared memory, before the wait for
 // the preceding kernel) and shared by its eight rows.  MODE 0: fp32 row-major;
-// 1: fp16 row-major; 2: fp16 in fragment order (frag_pos).
+// 1: fp16 row-major; 2: fp16 in fragment order (xt_pos).
 template <int MODE>
 __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x, int m, int k, uint64_t seed,
                                                   void* __restrict__ out) {
@@ -126,11 +131,10 @@ __global__ void __launch_bounds__(256) rht_kernel(const uint16_t* __restrict__ x
       dst[1] = make_uint4(f2_to_h2(v[8], v[9]), f2_to_h2(v[10], v[11]), f2_to_h2(v[12], v[13]),
                           f2_to_h2(v[14], v[15]));
     } else if (MODE == 2) {
-      uint16_t* rowp = reinterpret_cast<uint16_t*>(out) + (size_t)row * k;
 #pragma unroll
       for (int r4 = 0; r4 < 4; ++r4) {
         const int kk = blk * 512 + lane * 16 + 4 * r4;
-        *reinterpret_cast<uint2*>(rowp + frag_pos(kk)) =
+        *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + xt_pos(row, kk, k)) =
             make_uint2(f2_to_h2(v[4 * r4], v[4 * r4 + 1]), f2_to_h2(v[4 * r4 + 2], v[4 * r4 + 3]));
       }
     } else {
@@ -155,7 +159,7 @@ __global__ void __launch_bounds__(256) frag_permute_kernel(const uint16_t* __res
        i += (long long)gridDim.x * blockDim.x) {
     const long long row = i / (k / 4);
     const int kk = (int)(i - row * (k / 4)) * 4;
-    *reinterpret_cast<uint2*>(out + row * k + frag_pos(kk)) = *reinterpret_cast<const uint2*>(x + row * k + kk);
+    *reinterpret_cast<uint2*>(out + xt_pos((int)row, kk, k)) = *reinterpret_cast<const uint2*>(x + row * k + kk);
   }
 }
 

@@ -128,11 +128,10 @@ __device__ __forceinline__ void stackn_rht(const DmmaParams& p, const DmmaParams
     }
     wht512_warp(v);
     const float inv = 0.044194173824159216f;  // 1/sqrt(512)
-    uint16_t* row = xq + (size_t)t * p.k;
 #pragma unroll
     for (int r4 = 0; r4 < 4; ++r4) {
       const int kk = blk * 512 + lane * 16 + 4 * r4;
-      *reinterpret_cast<uint2*>(row + frag_pos(kk)) =
+      *reinterpret_cast<uint2*>(xq + xt_pos(t, kk, p.k)) =
           make_uint2(f2_to_h2(v[4 * r4] * inv, v[4 * r4 + 1] * inv), f2_to_h2(v[4 * r4 + 2] * inv, v[4 * r4 + 3] * inv));
     }
   }
