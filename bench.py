@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 import tqsynth  # noqa: E402
 
 PERSISTENT_MAX_M = 16  # tq_layer_stack runs one persistent kernel up to this many tokens
+REGISTER_DECODE_MAX_M = 32  # up to this many tokens the phases use the register-decode kernel, tcgen05 above
 METRIC = "decode-GEMV compressed-weight GB/s (% of HBM peak); layer-stack tokens/s at batch 1"
 
 WORKLOADS = {
@@ -576,7 +577,7 @@ def main():
                       "unit": "GB/s", "frac": bytes_step_layer / (kern_ms_layer * 1e-3) / 1e9 / hbm,
                       "traffic": None, "peak_source": peak_src,
                       "kernel": "rht_kernel + dmma_kernel (mma.sync register decode), all 4 phases",
-                      "phase_ms": ph_ms, "phase_bytes": pb} if m < 32 else
+                      "phase_ms": ph_ms, "phase_bytes": pb} if m <= REGISTER_DECODE_MAX_M else
                      {"bound": "tensor", "achieved": tensor_tflops, "peak": tflops, "unit": "TFLOP/s",
                       "frac": tensor_tflops / tflops, "traffic": None, "peak_source": peak_src,
                       "kernel": "rht_kernel + umma_kernel (tcgen05 decode-to-smem GEMM), all 4 phases",

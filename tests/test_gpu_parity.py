@@ -122,7 +122,7 @@ def test_gemv_deterministic_and_counters_reset(tq, torch_cuda):
 
 # ---- small-batch GEMM -------------------------------------------------------------
 
-@pytest.mark.parametrize("m", [2, 7, 8, 16, 17, 24, 31, 33, 64, 100])
+@pytest.mark.parametrize("m", [2, 7, 8, 16, 17, 24, 31, 32, 33, 64, 100])
 def test_gemm_small_batch(tq, torch_cuda, m):
     import torch
     n, k = 1040, 1536

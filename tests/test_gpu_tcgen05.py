@@ -1,4 +1,4 @@
-"""The decode-to-shared-memory tcgen05 GEMM (tq_gemm at m >= 32) against the
+"""The decode-to-shared-memory tcgen05 GEMM (tq_gemm at m >= 33) against the
 oracle: tile shapes with split-k, ragged rows and several token tiles."""
 import numpy as np
 import pytest
