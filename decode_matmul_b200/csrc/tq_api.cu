@@ -167,6 +167,41 @@ int dmma_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream, bool dry_run)
   return launch(kern, dim3((unsigned)grid), dim3(tq::DMMA_THREADS), smem, stream, p);
 }
 
+// Units per warp from which the two-row-tile kernel is used (measured at 32
+// tokens: 5.1 and more faster, e.g. 34816 x 5120 58 vs 68 us; 4.3 even;
+// 2.6 and fewer slower, e.g. 4096 x 4096 25 vs 21 us).
+constexpr int kDmma2MinUnits = 5;
+
+// The two-row-tile kernel (17-32 tokens): 32-row tiles, 8 warps per CTA.
+// Its partial sums take 32 x MC floats per warp and slot; the active warps
+// are capped at half the 16-row unit count so they fit the workspace that
+// dmma_ws_layout sizes for the 16-row kernel.
+template <int LV, int NT>
+int dmma2_launch_t(DmmaParams& p, int num_sms, cudaStream_t stream, bool dry_run) {
+  auto kern = tq::dmma_kernel_r2<LV, NT>;
+  const size_t smem = 16384u << LV;
+  static int occ_cache[kMaxDevices];
+  int dev = 0;
+  TQ_CUDA(cudaGetDevice(&dev));
+  int occ = occ_cache[dev];
+  if (occ == 0) {
+    TQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    TQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, tq::DMMA2_THREADS, smem));
+    if (occ < 1) return TQ_ERR_SHAPE;
+    occ_cache[dev] = occ;
+  }
+  if (dry_run) return TQ_OK;
+  const int64_t units16 = p.units;  // 16-row units (the workspace layout's count)
+  p.tiles = (p.n_total + 31) / 32;
+  p.units = (int64_t)p.tiles * p.blocks;
+  int64_t aw = (int64_t)num_sms * occ * tq::DMMA2_WARPS;
+  if (aw > p.units) aw = p.units;
+  if (aw > units16 / 2) aw = units16 / 2 > 0 ? units16 / 2 : 1;
+  p.active_warps = (int32_t)aw;
+  const int64_t grid = (aw + tq::DMMA2_WARPS - 1) / tq::DMMA2_WARPS;
+  return launch(kern, dim3((unsigned)grid), dim3(tq::DMMA2_THREADS), smem, stream, p);
+}
+
 template <int NT, bool HILO>
 int dmma_launch_lv(DmmaParams& p, int lv, int num_sms, cudaStream_t stream, bool dry_run) {
   switch (lv) {
@@ -200,7 +235,19 @@ int dmma_run(DmmaParams& p, bool hilo, void* ws, size_t ws_bytes, int num_sms, c
   switch (nt) {
     case 1: return dmma_launch_lv<1, false>(p, lv, num_sms, stream, dry_run);
     case 2: return dmma_launch_lv<2, false>(p, lv, num_sms, stream, dry_run);
-    default: return dmma_launch_lv<4, false>(p, lv, num_sms, stream, dry_run);
+    default:
+      // 17-32 tokens: two 16-row tiles per warp (x' loaded once for both)
+      // where that gives each of its warps at least kDmma2MinUnits 32-row
+      // units; on smaller shapes (few units per warp, most tiles split across
+      // warps) 16 warps of one row tile measured faster
+      if ((int64_t)((p.n_total + 31) / 32) * p.blocks < (int64_t)kDmma2MinUnits * num_sms * tq::DMMA2_WARPS)
+        return dmma_launch_lv<4, false>(p, lv, num_sms, stream, dry_run);
+      switch (lv) {
+        case 3: return dmma2_launch_t<3, 4>(p, num_sms, stream, dry_run);
+        case 2: return dmma2_launch_t<2, 4>(p, num_sms, stream, dry_run);
+        case 1: return dmma2_launch_t<1, 4>(p, num_sms, stream, dry_run);
+        default: return dmma2_launch_t<0, 4>(p, num_sms, stream, dry_run);
+      }
   }
 }
 

@@ -638,4 +638,289 @@ __global__ void __launch_bounds__(DMMA_THREADS, 1) dmma_kernel(const __grid_cons
   dmma_units<LV, NT, HILO>(p, smem, xs, W, c, lane);
 }
 
+// ---- two row tiles per warp (17-32 tokens) ------------------------------------
+//
+// At 17-32 tokens (four 8-token column tiles) the unit loop above spends as
+// many L1 wavefronts on x' as on the codebook gathers: every 16-row unit loads
+// its 16 KB of x' again.  Here a warp's unit is 32 rows x one 256-weight block:
+// lane (g, q) decodes rows g, g+8, g+16 and g+24, and both 16-row MMA tiles
+// use the same x' registers, so x' costs half as many wavefronts per weight.
+// The extra registers (codes, scales and accumulators of two more rows) do not
+// fit 16 warps at 128 registers each, so this kernel runs 8 warps per SM with
+// up to 255 registers.  Tiles are 32 rows; a tile split across warps is summed
+// by the last warp to arrive, in warp order.  Batch 1 and the persistent stack
+// kernels keep the 16-row loop above.
+constexpr int DMMA2_WARPS = 8;
+constexpr int DMMA2_THREADS = DMMA2_WARPS * 32;
+
+struct DmmaRows2 {
+  const uint8_t* c[4];  // code bytes of rows g + 8 i, chunk q, block 0
+  const uint16_t* s[4]; // their scales
+};
+
+struct DmmaChunk2 {
+  uint4 c[4];
+  uint32_t s[4];
+};
+
+__device__ __forceinline__ DmmaRows2 dmma2_rows(const DmmaParams& p, int t, int g, int q) {
+  DmmaRows2 r;
+  const int gpr = p.k >> 2;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = min(t * 32 + g + 8 * i, p.n_total - 1);  // rows past the end are clamped, never stored
+    const uint8_t* c;
+    const uint16_t* sc;
+    int l;
+    seg_lookup(p, row, c, sc, l);
+    r.c[i] = c + (size_t)l * gpr + q * 16;
+    r.s[i] = sc + (size_t)l * p.blocks;
+  }
+  return r;
+}
+
+// Codes of block b, scales from the scale-pair words (see dmma_fetch).
+__device__ __forceinline__ DmmaChunk2 dmma2_fetch(const DmmaRows2& r, int b, uint32_t (&sp)[4], bool fresh) {
+  DmmaChunk2 ch;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ch.c[i] = ldg_stream_u4(r.c[i] + b * 64);
+  if (fresh || (b & 1) == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sp[i] = __ldg(reinterpret_cast<const uint32_t*>(r.s[i] + (b & ~1)));
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) ch.s[i] = (b & 1) ? (sp[i] >> 16) : (sp[i] & 0xFFFFu);
+  return ch;
+}
+
+// Element of a 32-row x MC partial for accumulator value (h, jt, i) of lane (g, q).
+template <int NT>
+__device__ __forceinline__ int dmma2_pidx(int g, int q, int h, int jt, int i) {
+  constexpr int MC = NT * 8;
+  return (16 * h + g + ((i < 2) ? 0 : 8)) * MC + jt * 8 + 2 * q + (i & 1);
+}
+
+template <int NT>
+__device__ __forceinline__ void dmma2_epilogue(const DmmaParams& p, int t, int g, int q, const float (&v)[2][NT][4]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tok = jt * 8 + 2 * q + (i & 1);
+        const int row = t * 32 + 16 * h + g + ((i < 2) ? 0 : 8);
+        if (tok < p.m && row < p.n_total) {
+          const float y = v[h][jt][i];
+          if (p.y) p.y[(size_t)tok * p.n_total + row] = y;
+          if (row < p.handoff_rows) p.handoff[(size_t)tok * p.handoff_rows + row] = f_to_bf16_bits(p.alpha * y);
+        }
+      }
+}
+
+template <int NT>
+__device__ __forceinline__ void dmma2_write_partial(const DmmaParams& p, int64_t W, int slot, int g, int q,
+                                                    const float (&acc)[2][NT][4]) {
+  constexpr int MC = NT * 8;
+  float* part = p.partials + ((size_t)W * 2 + slot) * (32 * MC);
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) part[dmma2_pidx<NT>(g, q, h, jt, i)] = acc[h][jt][i];
+}
+
+// The last contributor of tile t sums every contributor's partial in warp order.
+template <int NT>
+__device__ __forceinline__ void dmma2_reduce_tile(const DmmaParams& p, int t, int g, int q) {
+  constexpr int MC = NT * 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t t0 = (int64_t)t * p.blocks, t1 = t0 + p.blocks;
+  const int64_t wa = dmma_warp_of(t0, p.units, p.active_warps);
+  const int64_t wz = dmma_warp_of(t1 - 1, p.units, p.active_warps);
+  __threadfence();
+  const int first_slot = (dmma_warp_begin(wa, p.units, p.active_warps) >= t0) ? 0 : 1;
+  float sum[2][NT][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sum[h][jt][i] = 0.f;
+  for (int64_t w = wa; w <= wz; ++w) {
+    const int s = (w == wa) ? first_slot : 0;
+    const float* src = p.partials + ((size_t)w * 2 + s) * (32 * MC);
+    float v[2][NT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[h][jt][i] = __ldcg(src + dmma2_pidx<NT>(g, q, h, jt, i));
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum[h][jt][i] += v[h][jt][i];
+  }
+  dmma2_epilogue<NT>(p, t, g, q, sum);
+  if (lane == 0) p.counters[t] = 0;  // leave the counter ready for the next call
+}
+
+template <int NT>
+__device__ __forceinline__ void dmma2_publish(const DmmaParams& p, int64_t W, int g, int q, bool has_head, int head_t,
+                                              const float (&hacc)[2][NT][4], bool has_tail, int tail_t, int tail_slot,
+                                              const float (&tacc)[2][NT][4]) {
+  const int lane = threadIdx.x & 31;
+  if (has_head) dmma2_write_partial<NT>(p, W, 0, g, q, hacc);
+  if (has_tail) dmma2_write_partial<NT>(p, W, tail_slot, g, q, tacc);
+  __threadfence();
+  __syncwarp();
+  int oh = 0, ot = 0;
+  if (lane == 0) {
+    if (has_head) oh = atomicAdd(p.counters + head_t, 1);
+    if (has_tail) ot = atomicAdd(p.counters + tail_t, 1);
+  }
+  oh = __shfl_sync(0xffffffffu, oh, 0);
+  ot = __shfl_sync(0xffffffffu, ot, 0);
+  if (has_head && oh == dmma_contributors(p, head_t) - 1) dmma2_reduce_tile<NT>(p, head_t, g, q);
+  if (has_tail && ot == dmma_contributors(p, tail_t) - 1) dmma2_reduce_tile<NT>(p, tail_t, g, q);
+}
+
+template <int LV, int NT>
+__device__ __forceinline__ void dmma2_units(const DmmaParams& p, const uint8_t* smem, int64_t W, int lane) {
+  constexpr int V = 1 << LV;
+  constexpr int SH = 3 + LV;
+  const int g = lane >> 2, q = lane & 3;
+  const bool active = W < p.active_warps;
+  const int64_t wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
+  const int64_t we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
+  if (wb >= we) return;
+  int t = (int)(wb / p.blocks), b = (int)(wb - (int64_t)t * p.blocks);
+  DmmaRows2 rows = dmma2_rows(p, t, g, q);
+  uint32_t sp[4];
+  DmmaChunk2 cur = dmma2_fetch(rows, b, sp, true);
+  const uint32_t vofs = (uint32_t)((lane & (V - 1)) << 3);
+  const int jt_last = (p.m - 1) >> 3;  // column tiles past it re-read it (their outputs are discarded)
+  float acc[2][NT][4], hacc[2][NT][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[h][jt][i] = hacc[h][jt][i] = 0.f;
+  bool has_head = false, has_tail = false;
+  int head_t = 0, tail_t = 0;
+  const int nunits = (int)(we - wb);
+  for (int iu = 0; iu < nunits; ++iu) {
+    int tn = t, bn = b + 1;
+    if (bn == p.blocks) {
+      bn = 0;
+      ++tn;
+    }
+    DmmaRows2 nrows = rows;
+    DmmaChunk2 nxt;
+    if (iu + 1 < nunits) {
+      if (bn == 0) nrows = dmma2_rows(p, tn, g, q);
+      nxt = dmma2_fetch(nrows, bn, sp, false);
+    }
+    const uint16_t* xg_lane[NT];
+#pragma unroll
+    for (int jt = 0; jt < NT; ++jt)  // step pair 0 of block b, tokens of column tile jt (xt_pos)
+      xg_lane[jt] = p.x_f16 + (size_t)min(jt, jt_last) * 8 * p.k + (size_t)b * 2048 + lane * 8;
+    // previous code byte of each row chunk (state of code 0); 0 at a block start
+    uint32_t pv[4], s2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      pv[i] = __shfl_up_sync(0xffffffffu, cur.c[i].w, 1) >> 24;
+      if (q == 0) pv[i] = 0;
+      s2[i] = cur.s[i] | (cur.s[i] << 16);
+    }
+    uint4 bpair[NT];
+#pragma unroll
+    for (int i4 = 0; i4 < 4; ++i4) {
+      uint32_t off[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t w4[4] = {cur.c[i].x, cur.c[i].y, cur.c[i].z, cur.c[i].w};
+        const uint32_t r = __byte_perm(w4[i4], 0, 0x0123);
+        const uint32_t hp = (i4 == 0) ? pv[i] : __byte_perm(w4[i4 > 0 ? i4 - 1 : 0], 0, 0x0123);
+        word_offsets<SH>(r, hp, vofs, off[i]);
+      }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int j = i4 * 4 + jj;
+        uint32_t a[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint2 ea = *reinterpret_cast<const uint2*>(smem + off[2 * h][jj]);
+          const uint2 eb = *reinterpret_cast<const uint2*>(smem + off[2 * h + 1][jj]);
+          a[h][0] = hmul2_u32(ea.x, s2[2 * h]);
+          a[h][2] = hmul2_u32(ea.y, s2[2 * h]);
+          a[h][1] = hmul2_u32(eb.x, s2[2 * h + 1]);
+          a[h][3] = hmul2_u32(eb.y, s2[2 * h + 1]);
+        }
+        // one 16-byte load holds this lane's quads of steps j and j + 1
+        if ((j & 1) == 0) {
+#pragma unroll
+          for (int jt = 0; jt < NT; ++jt) bpair[jt] = __ldg(reinterpret_cast<const uint4*>(xg_lane[jt] + 128 * j));
+        }
+#pragma unroll
+        for (int jt = 0; jt < NT; ++jt) {
+          const uint32_t b0 = (j & 1) ? bpair[jt].z : bpair[jt].x, b1 = (j & 1) ? bpair[jt].w : bpair[jt].y;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) mma_16816(acc[h][jt], a[h], b0, b1);
+        }
+      }
+    }
+    if (iu + 1 == nunits || bn == 0) {  // tile t ends here (for this warp)
+      const int64_t t0 = (int64_t)t * p.blocks;
+      if (t0 >= wb && t0 + p.blocks <= we) {
+        dmma2_epilogue<NT>(p, t, g, q, acc);  // the whole tile ran in this warp
+      } else if (iu + 1 < nunits) {
+        has_head = true;  // the range's first tile, shared with earlier warps: published at the end
+        head_t = t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hacc[h][jt][i] = acc[h][jt][i];
+      } else {
+        has_tail = true;
+        tail_t = t;
+      }
+      if (iu + 1 < nunits) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int jt = 0; jt < NT; ++jt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[h][jt][i] = 0.f;
+      }
+    }
+    t = tn;
+    b = bn;
+    rows = nrows;
+    cur = nxt;
+  }
+  if (has_head || has_tail) {
+    const int tail_slot = (tail_t == (int)(wb / p.blocks)) ? 0 : 1;  // slot 0 holds the range's first tile
+    dmma2_publish<NT>(p, W, g, q, has_head, head_t, hacc, has_tail, tail_t, tail_slot, acc);
+  }
+}
+
+template <int LV, int NT>
+__global__ void __launch_bounds__(DMMA2_THREADS, 1) dmma_kernel_r2(const __grid_constant__ DmmaParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
+  build_views<LV>(smem, p.codebook, tid, DMMA2_THREADS);  // no kernel of the stream writes the codebook
+  pdl_wait();
+  __syncthreads();
+  dmma2_units<LV, NT>(p, smem, (int64_t)blockIdx.x * DMMA2_WARPS + warp, lane);
+}
+
 }  // namespace tq

@@ -136,6 +136,27 @@ def test_gemm_small_batch(tq, torch_cuda, m):
     assert err < TOL, err
 
 
+@pytest.mark.parametrize("m", [24, 32])
+def test_gemm_two_row_tiles(tq, torch_cuda, m):
+    # 17-32 tokens on a shape with enough 32-row units for the two-row-tile
+    # kernel (at least 5 per warp of 148 x 8): 297 tiles x 20 blocks, the last
+    # tile 8 rows of 32; every tile spans about four warps, so each is summed
+    # from partials.  Compared element by element on every row of the first 8
+    # tiles, 8 tiles in the middle and the ragged last tile (the whole matrix
+    # would take the oracle ~15 s).
+    import torch
+    n, k = 9480, 5120
+    hw = host_weight(4, 0, 6, n, k)
+    x = tqsynth.activations(4, m, k)
+    xr = f16_exact(oracle.rht(x, m, k, 5))
+    xd = torch.from_numpy(xr.astype(np.float16)).cuda()
+    y = tq.tq_gemm(dev_weight(hw), xd).cpu().numpy()
+    for r0, r1 in [(0, 256), (4736, 4992), (n - 8, n)]:
+        want = oracle.linear_rows(hw.codes, hw.scales, hw.codebook, k, xr, m, r0, r1)
+        err = oracle.rel_err(y[:, r0:r1], want)
+        assert err < TOL, (r0, err)
+
+
 # ---- layer phases ------------------------------------------------------------------
 
 SMALL = tqsynth.StackShape("small", 2, 512, 1024, 512, 1536)
