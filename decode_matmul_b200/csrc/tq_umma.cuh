@@ -18,17 +18,17 @@
 //               operand; then the epilogue (tcgen05.ld), warps 4-7 and 8-11
 //               taking one half of the columns each
 // Where A lives depends on the tile width:
-//   * up to 128 tokens, in shared memory (the K-major 128B-swizzled tile);
-//     at 64 tokens the stage ring is 6 deep, which measured 15% faster than
-//     4 on the 27B-class gate|up shape at 32 tokens: the loop is bound by
-//     the latency of the stage round trip (TMA in, decode, MMA, release),
-//     not by shared-memory bandwidth;
-//   * at 256 tokens, in tensor memory (tcgen05.st by the decoders; row r of
-//     the tile in TMEM lane r, the fp16 pair (2c, 2c+1) of the k step in
-//     column c of the stage), because there the loop is bound by shared
-//     memory and a decoded tile in shared memory costs a 16 KB write and a
-//     16 KB MMA read per k step (9% faster on the Qwen3-4B gate|up shape at
-//     512 tokens).
+//   * at 64 and 256 tokens, in tensor memory (tcgen05.st by the decoders; row
+//     r of the tile in TMEM lane r, the fp16 pair (2c, 2c+1) of the k step in
+//     column c of the stage).  At 256 tokens the loop is bound by shared
+//     memory, where a decoded tile costs a 16 KB write and a 16 KB MMA read
+//     per k step (without them: 16% faster on the Qwen3-4B gate|up shape at
+//     512 tokens).  At 64 tokens the loop is bound by the latency of the
+//     stage round trip (TMA in, decode, MMA, release); A out of shared memory
+//     leaves room for 12 stages of 10 KB (6 stages of 26 KB with A in shared
+//     memory were 15% faster than 4 on the 27B-class gate|up shape at 32
+//     tokens, 12 in TMEM another 4-5% at 64 tokens);
+//   * at 128 tokens, in shared memory (the K-major 128B-swizzled tile).
 // Stages are handed over with mbarriers; every wait is bounded and, when it
 // runs out, the kernel records TQ_ERR_TIMEOUT in the status word and drains.
 #pragma once
@@ -179,10 +179,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 template <int BN>
 struct UmmaSmem {
-  // A in tensor memory at 256 tokens (see the file header)
-  static constexpr bool TMEM_A = BN == 256;
-  // stages: 6 at 64 tokens, 4 above; the codebook as 4 views (64 KB)
-  static constexpr int STAGES = BN == 64 ? 6 : 4;
+  // A in tensor memory at 64 and 256 tokens (see the file header)
+  static constexpr bool TMEM_A = BN != 128;
+  // stages: 12 at 64 tokens, 4 above; the codebook as 4 views (64 KB)
+  static constexpr int STAGES = BN == 64 ? 12 : 4;
   static constexpr int LV = 2;
   // TMEM columns: the fp32 accumulator [0, BN), then (TMEM_A) 32 per stage
   static constexpr uint32_t A_COL0 = BN;

@@ -172,9 +172,9 @@ TQ_API int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes);
  * tokens.  x_rot_f16_d: device fp16 [m][k] (tq_rht with TQ_F16), 16-byte
  * aligned.  y_d: device fp32 [m][n], 16-byte aligned.  The kernel is chosen by
  * m: register-decode warp MMAs up to 32 tokens, tcgen05 MMAs with TMEM
- * accumulators from 33 (the decoded weights staged in shared memory up to 128
- * tokens per tile, in tensor memory at 256).  Same workspace rules as
- * tq_gemv.
+ * accumulators from 33 (the decoded weights staged in tensor memory for
+ * 64- and 256-token tiles, in shared memory for 128-token tiles).  Same
+ * workspace rules as tq_gemv.
  * m == 0 returns TQ_OK without a launch; m > 4096 is TQ_ERR_SHAPE. */
 TQ_API int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
             size_t ws_bytes, void* stream);
