@@ -26,7 +26,7 @@ EXPORTS = ("tq_pack_info", "tq_decode", "tq_rht", "tq_gemv_workspace", "tq_gemv"
            "tq_workspace_init", "tq_stack_phase_seed", "tq_layer_phase_workspace", "tq_layer_stack_workspace",
            "tq_layer_phase", "tq_layer_stack", "tq_status_string", "tq_last_cuda_error", "tq_gemv_noalloc",
            "tq_layer_stack_buffers", "tq_layer_stack_outputs", "tq_encode", "tq_ldlq_workspace", "tq_ldlq_encode",
-           "tq_layer_stack_ex", "tq_workspace_status")
+           "tq_layer_stack_ex", "tq_workspace_status", "tq_gemm_ex")
 TQ_STATUS_OFFSET = 65532
 TQ_GEMV_MAX_K = 53760
 
@@ -82,6 +82,7 @@ def _lib():
             "tq_gemv_noalloc": ([W, vp, vp, vp], ctypes.c_int),
             "tq_gemm_workspace": ([i32, i32, i32, szp], ctypes.c_int),
             "tq_gemm": ([W, vp, i32, vp, vp, sz, vp], ctypes.c_int),
+            "tq_gemm_ex": ([W, vp, i32, vp, vp, sz, ctypes.POINTER(tq_stack_options_t), vp], ctypes.c_int),
             "tq_workspace_init": ([vp, sz, vp], ctypes.c_int),
             "tq_stack_phase_seed": ([u64, i32, i32], u64),
             "tq_layer_phase_workspace": ([LY, i32, i32, szp], ctypes.c_int),
@@ -229,6 +230,17 @@ def tq_gemm(w: DeviceWeight, x_rot_f16, y=None, ws=None, stream=None):
     s = w.struct()
     _ok(_lib().tq_gemm(ctypes.byref(s), _ptr(x_rot_f16), m, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
         "tq_gemm")
+    return y
+
+
+def tq_gemm_ex(w: DeviceWeight, x_rot_f16, y, ws, spin_limit: int = 0, test_skip_arrive: int = -1, stream=None):
+    """tq_gemm with options: the tcgen05 kernel's poll limit (0 = the default)
+    and its timeout test hook (a thread block whose MMA wait runs out; -1 =
+    off).  Both act from 33 tokens on."""
+    opt = tq_stack_options_t(spin_limit, test_skip_arrive)
+    s = w.struct()
+    _ok(_lib().tq_gemm_ex(ctypes.byref(s), _ptr(x_rot_f16), x_rot_f16.shape[0], _ptr(y), _ptr(ws), ws.numel(),
+                          ctypes.byref(opt), _stream(stream)), "tq_gemm_ex")
     return y
 
 

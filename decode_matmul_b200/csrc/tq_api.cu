@@ -347,7 +347,8 @@ int umma_launch_t(tq::UmmaParams& p, int grid, cudaStream_t stream) {
 // k and the codebook.  x_f16: device fp16 [m][k].
 int umma_run(const uint8_t* const* codes, const uint16_t* const* scales, const int32_t* rows, int nseg,
              const uint16_t* codebook, int32_t k, int32_t m, const uint16_t* x_f16, float* y, uint16_t* handoff,
-             float alpha, void* ws, size_t ws_bytes, cudaStream_t stream) {
+             float alpha, void* ws, size_t ws_bytes, cudaStream_t stream, const tq_stack_options_t* opt = nullptr) {
+  if (opt && opt->test_skip_arrive < -1) return TQ_ERR_VALUE;
   int st = get_encode_tiled();
   if (st != TQ_OK) return st;
   int64_t n_total = 0;
@@ -385,7 +386,8 @@ int umma_run(const uint8_t* const* codes, const uint16_t* const* scales, const i
   p.row_tiles = u.row_tiles;
   p.tok_tiles = u.tok_tiles;
   p.splits = u.splits;
-  p.spin_limit = 1u << 21;  // try_wait polls; far above any healthy wait
+  p.spin_limit = (opt && opt->spin_limit) ? opt->spin_limit : 1u << 21;  // try_wait polls; far above any healthy wait
+  p.skip_arrive_cta = opt ? opt->test_skip_arrive : -1;
   const int grid = u.row_tiles * u.tok_tiles * u.splits;
   switch (u.bn) {
     case 64: return umma_launch_t<64>(p, grid, stream);
@@ -607,6 +609,12 @@ int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes) {
 
 int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
             size_t ws_bytes, void* stream) {
+  return tq_gemm_ex(w, x_rot_f16_d, m, y_d, workspace_d, ws_bytes, nullptr, stream);
+}
+
+int tq_gemm_ex(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
+               size_t ws_bytes, const tq_stack_options_t* options, void* stream) {
+  if (options && options->test_skip_arrive < -1) return TQ_ERR_VALUE;
   int st = check_weight(w);
   if (st != TQ_OK) return st;
   if (m < 0 || m > 4096) return TQ_ERR_SHAPE;
@@ -621,7 +629,7 @@ int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float*
     const uint16_t* sc = w->scales_d;
     const int32_t rows = w->n;
     return umma_run(&c, &sc, &rows, 1, w->codebook_d, w->k, m, x_rot_f16_d, y_d, nullptr, 0.f, workspace_d, ws_bytes,
-                    (cudaStream_t)stream);
+                    (cudaStream_t)stream, options);
   }
   // the small-batch kernel reads x' in fragment order: permute it into the
   // workspace after the matmul scratch

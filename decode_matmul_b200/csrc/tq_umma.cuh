@@ -64,6 +64,8 @@ struct UmmaParams {
   int32_t* status;     // error word or null
   int32_t row_tiles, tok_tiles, splits;
   uint32_t spin_limit;  // bounded waits
+  int32_t skip_arrive_cta;  // timeout test hook: this CTA's decoded-stage barriers expect one arrival
+                            // too many, so its MMA wait runs out (-1 = off)
 };
 
 // ---- PTX wrappers -------------------------------------------------------------
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     *abort_flag = 0;
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_dec + 8 * s, UM_DEC_THREADS);
+      mbar_init(bar_dec + 8 * s, UM_DEC_THREADS + ((int)blockIdx.x == p.skip_arrive_cta ? 1 : 0));
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_acc, 1);
@@ -480,9 +482,12 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     }
   }
 
-  if (*abort_flag && tid == 0 && p.status) atomicExch(p.status, UM_TIMEOUT_STATUS);
   tc_fence_before();
   __syncthreads();
+  // after the barrier: every role has set the flag by now if its wait ran out
+  // (a producer with no more k steps than stages never waits, and would
+  // otherwise read the flag before the MMA thread sets it)
+  if (*abort_flag && tid == 0 && p.status) atomicExch(p.status, UM_TIMEOUT_STATUS);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(L::TMEM_COLS));

@@ -179,6 +179,19 @@ TQ_API int tq_gemm_workspace(int32_t n, int32_t k, int32_t m, size_t* bytes);
 TQ_API int tq_gemm(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
             size_t ws_bytes, void* stream);
 
+/* tq_gemm with options (tq_stack_options_t, declared with tq_layer_stack_ex;
+ * NULL = the defaults, which is tq_gemm).  They act on the tcgen05 kernel
+ * (m >= 33) only: spin_limit = try-wait polls of each of its bounded mbarrier
+ * waits (0 = the default, 2^21); test_skip_arrive = c >= 0 makes thread block
+ * c's decoded-stage barriers expect one arrival more than its decoders make,
+ * so that block's MMA wait runs out: the launch ends with TQ_ERR_TIMEOUT in
+ * the workspace's status word and undefined outputs (a test hook of the
+ * timeout path; -1 = off, below -1 = TQ_ERR_VALUE).  The register-decode
+ * kernel (m <= 32) has no wait on other thread blocks and ignores them. */
+typedef struct tq_stack_options tq_stack_options_t;
+TQ_API int tq_gemm_ex(const tq_weight_t* w, const uint16_t* x_rot_f16_d, int32_t m, float* y_d, void* workspace_d,
+                      size_t ws_bytes, const tq_stack_options_t* options, void* stream);
+
 /* Zero a workspace (cudaMemsetAsync on `stream`). */
 TQ_API int tq_workspace_init(void* workspace_d, size_t bytes, void* stream);
 
@@ -265,10 +278,10 @@ TQ_API int tq_layer_stack(const tq_layer_t* layers, int32_t n_layers, const uint
  *   word and undefined outputs.  Values below -1 are TQ_ERR_VALUE; a block
  *   index past the grid makes nothing happen.  Ignored by the per-phase path
  *   (m > 16). */
-typedef struct tq_stack_options {
+struct tq_stack_options {
   uint32_t spin_limit;
   int32_t test_skip_arrive;
-} tq_stack_options_t;
+};
 
 /* tq_layer_stack with options (NULL = the defaults, which is tq_layer_stack). */
 TQ_API int tq_layer_stack_ex(const tq_layer_t* layers, int32_t n_layers, const uint16_t* h_in_bf16_d, int32_t m,

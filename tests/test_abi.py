@@ -126,6 +126,8 @@ def test_gemv_k_limit_and_new_entry_points_checks():
     arr = (tq.tq_layer_t * 1)(*layers)
     opt = tq.tq_stack_options_t(0, -2)
     assert L.tq_layer_stack_ex(arr, 1, 16, 1, 0, 16, 16, 1 << 30, ctypes.byref(opt), None) == tq.TQ_ERR_VALUE
+    w = tq.tq_weight_t(16, 16, 16, 1024, 1536)
+    assert L.tq_gemm_ex(ctypes.byref(w), 16, 64, 16, 16, 1 << 30, ctypes.byref(opt), None) == tq.TQ_ERR_VALUE
 
 
 def test_stack_phase_seed_matches_oracle():
