@@ -789,19 +789,41 @@ __device__ __forceinline__ void dmma2_publish(const DmmaParams& p, int64_t W, in
   if (has_tail && ot == dmma_contributors(p, tail_t) - 1) dmma2_reduce_tile<NT>(p, tail_t, g, q);
 }
 
+// Units [wb, we) of warp W and its first chunk of codes (loaded ahead: the
+// weights never depend on activations).
+struct DmmaCursor2 {
+  int64_t wb, we;
+  int t, b;
+  DmmaRows2 rows;
+  DmmaChunk2 cur;
+  uint32_t sp[4];
+};
+
+__device__ __forceinline__ void dmma2_begin(const DmmaParams& p, int64_t W, int g, int q, DmmaCursor2& c) {
+  const bool active = W < p.active_warps;
+  c.wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
+  c.we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
+  c.t = c.b = 0;
+  if (c.wb < c.we) {
+    c.t = (int)(c.wb / p.blocks);
+    c.b = (int)(c.wb - (int64_t)c.t * p.blocks);
+    c.rows = dmma2_rows(p, c.t, g, q);
+    c.cur = dmma2_fetch(c.rows, c.b, c.sp, true);
+  }
+}
+
 template <int LV, int NT>
-__device__ __forceinline__ void dmma2_units(const DmmaParams& p, const uint8_t* smem, int64_t W, int lane) {
+__device__ __forceinline__ void dmma2_units(const DmmaParams& p, const uint8_t* smem, int64_t W, int lane,
+                                            DmmaCursor2& c) {
   constexpr int V = 1 << LV;
   constexpr int SH = 3 + LV;
   const int g = lane >> 2, q = lane & 3;
-  const bool active = W < p.active_warps;
-  const int64_t wb = active ? dmma_warp_begin(W, p.units, p.active_warps) : 0;
-  const int64_t we = active ? dmma_warp_begin(W + 1, p.units, p.active_warps) : 0;
+  const int64_t wb = c.wb, we = c.we;
   if (wb >= we) return;
-  int t = (int)(wb / p.blocks), b = (int)(wb - (int64_t)t * p.blocks);
-  DmmaRows2 rows = dmma2_rows(p, t, g, q);
-  uint32_t sp[4];
-  DmmaChunk2 cur = dmma2_fetch(rows, b, sp, true);
+  int t = c.t, b = c.b;
+  DmmaRows2 rows = c.rows;
+  uint32_t sp[4] = {c.sp[0], c.sp[1], c.sp[2], c.sp[3]};
+  DmmaChunk2 cur = c.cur;
   const uint32_t vofs = (uint32_t)((lane & (V - 1)) << 3);
   const int jt_last = (p.m - 1) >> 3;  // column tiles past it re-read it (their outputs are discarded)
   float acc[2][NT][4], hacc[2][NT][4];
@@ -918,9 +940,12 @@ __global__ void __launch_bounds__(DMMA2_THREADS, 1) dmma_kernel_r2(const __grid_
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
   build_views<LV>(smem, p.codebook, tid, DMMA2_THREADS);  // no kernel of the stream writes the codebook
+  const int64_t W = (int64_t)blockIdx.x * DMMA2_WARPS + warp;
+  DmmaCursor2 c;
+  dmma2_begin(p, W, lane >> 2, lane & 3, c);  // weights: requested before waiting on the previous kernel
   pdl_wait();
   __syncthreads();
-  dmma2_units<LV, NT>(p, smem, (int64_t)blockIdx.x * DMMA2_WARPS + warp, lane);
+  dmma2_units<LV, NT>(p, smem, W, lane, c);
 }
 
 }  // namespace tq
