@@ -179,16 +179,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 // ---- shared-memory layout ---------------------------------------------------------
 
-template <int BN>
+// PAIR: two CTAs per SM (64-token tiles when there are at least as many
+// tiles as SMs): 6 stages, 2 codebook views and 256 TMEM columns each, so
+// that two fit one SM; every tile then runs in one wave, and the SM has two
+// independent stage pipelines for the latency-bound loop (27B-class gate|up
+// shape, 272 tiles, at 64 tokens: 75.9 -> 56.0 us).  With fewer tiles (split
+// k) the single-CTA form is faster.
+template <int BN, bool PAIR = false>
 struct UmmaSmem {
+  static_assert(!PAIR || BN == 64, "two CTAs per SM at 64-token tiles only");
   // A in tensor memory at 64 and 256 tokens (see the file header)
   static constexpr bool TMEM_A = BN != 128;
-  // stages: 12 at 64 tokens, 4 above; the codebook as 4 views (64 KB)
-  static constexpr int STAGES = BN == 64 ? 12 : 4;
-  static constexpr int LV = 2;
+  // stages: 12 at 64 tokens (6 in PAIR), 4 above; the codebook as 4 views
+  // (64 KB), 2 in PAIR
+  static constexpr int STAGES = PAIR ? 6 : (BN == 64 ? 12 : 4);
+  static constexpr int LV = PAIR ? 1 : 2;
   // TMEM columns: the fp32 accumulator [0, BN), then (TMEM_A) 32 per stage
   static constexpr uint32_t A_COL0 = BN;
-  static constexpr uint32_t TMEM_COLS = TMEM_A ? 512 : BN;
+  static constexpr uint32_t TMEM_COLS = PAIR ? 256 : (TMEM_A ? 512 : BN);
   static constexpr uint32_t A_BYTES = TMEM_A ? 0 : UM_BM * 128;  // 16 KB per stage in shared memory
   static constexpr uint32_t B_BYTES = BN * 128;        // BN rows of 64 fp16
   static constexpr uint32_t C_BYTES = UM_BM * 16;      // 16 code bytes per row
@@ -200,13 +208,14 @@ struct UmmaSmem {
   static constexpr uint32_t MISC_OFF = BAR_OFF + (3 * STAGES + 1) * 8;
   static constexpr uint32_t BYTES = MISC_OFF + 64;
   static constexpr uint32_t ALLOC = BYTES + 1024;  // slack to align the base to 1024
-  static_assert(ALLOC <= 227 * 1024, "shared memory per block");
+  static_assert(ALLOC <= (PAIR ? 113 : 227) * 1024, "shared memory per block");
   static_assert(!TMEM_A || A_COL0 + 32 * STAGES <= TMEM_COLS, "tensor memory columns");
 };
 
-template <int BN>
-__global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_constant__ UmmaParams p) {
-  using L = UmmaSmem<BN>;
+template <int BN, bool PAIR = false>
+__global__ void __launch_bounds__(UM_THREADS, PAIR ? 2 : 1) umma_kernel(const __grid_constant__ UmmaParams p) {
+  using L = UmmaSmem<BN, PAIR>;
+  const int splits = PAIR ? 1 : p.splits;  // the host never splits k in PAIR
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -214,7 +223,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // tile coordinates
-  const int tile = blockIdx.x / p.splits, split = blockIdx.x - tile * p.splits;
+  const int tile = blockIdx.x / splits, split = blockIdx.x - tile * splits;
   const int rt = tile / p.tok_tiles, tt = tile - rt * p.tok_tiles;
   const int row0 = rt * UM_BM, tok0 = tt * BN;
   int seg = 0;
@@ -222,8 +231,8 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
   if (p.nseg > 2 && row0 >= p.seg_row0[2]) seg = 2;
   const int seg_row = row0 - p.seg_row0[seg];
   const int blocks = p.k / 256;
-  const int b_lo = (int)((int64_t)split * blocks / p.splits);
-  const int b_hi = (int)((int64_t)(split + 1) * blocks / p.splits);
+  const int b_lo = (int)((int64_t)split * blocks / splits);
+  const int b_hi = (int)((int64_t)(split + 1) * blocks / splits);
   const int it0 = b_lo * 4, it1 = b_hi * 4;  // 64-wide k steps of this split
   const int niters = it1 - it0;
 
@@ -395,7 +404,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
     if (!ok) *abort_flag = 1;
     tc_fence_after();
     const int n = row0 + wq * 32 + lane;
-    float* part = p.partials + ((size_t)tile * p.splits + split) * (size_t)(BN * UM_BM);
+    float* part = p.partials + ((size_t)tile * splits + split) * (size_t)(BN * UM_BM);
     for (int c0 = half * (BN / 2); c0 < (half + 1) * (BN / 2); c0 += 32) {
       float v[32];
       if (ok) {
@@ -404,7 +413,7 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = 0.f;
       }
-      if (p.splits == 1) {
+      if (splits == 1) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int tok = tok0 + c0 + j;
@@ -418,16 +427,16 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
         for (int j = 0; j < 32; ++j) part[(size_t)(c0 + j) * UM_BM + wq * 32 + lane] = v[j];
       }
     }
-    if (p.splits > 1) {
+    if (splits > 1) {
       // the last split of this tile to finish sums all of them in split order,
       // 4 rows per float4, every epilogue thread in parallel
       __threadfence();
       asm volatile("bar.sync 1, 256;\n" ::: "memory");
       if (tid == 128) bcast[0] = atomicAdd(p.counters + tile, 1);
       asm volatile("bar.sync 1, 256;\n" ::: "memory");
-      if (bcast[0] == p.splits - 1) {
+      if (bcast[0] == splits - 1) {
         __threadfence();
-        const float4* tp = reinterpret_cast<const float4*>(p.partials + (size_t)tile * p.splits * (size_t)(BN * UM_BM));
+        const float4* tp = reinterpret_cast<const float4*>(p.partials + (size_t)tile * splits * (size_t)(BN * UM_BM));
         constexpr int Q = BN * UM_BM / 4;  // float4s per split tile
         const int et = tid - 128;
         for (int i0 = et; i0 < Q; i0 += 4 * UM_DEC_THREADS) {
@@ -436,19 +445,19 @@ __global__ void __launch_bounds__(UM_THREADS, 1) umma_kernel(const __grid_consta
           for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           // the loads of up to UM_SPLIT_BATCH splits are all in flight before
           // the first add (the sum is latency-bound otherwise)
-          for (int sp0 = 0; sp0 < p.splits; sp0 += UM_SPLIT_BATCH) {
+          for (int sp0 = 0; sp0 < splits; sp0 += UM_SPLIT_BATCH) {
             float4 v4[UM_SPLIT_BATCH][4];
 #pragma unroll
             for (int b = 0; b < UM_SPLIT_BATCH; ++b)
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 const int i = i0 + u * UM_DEC_THREADS;
-                v4[b][u] = (i < Q && sp0 + b < p.splits) ? __ldcg(tp + (size_t)(sp0 + b) * Q + i)
+                v4[b][u] = (i < Q && sp0 + b < splits) ? __ldcg(tp + (size_t)(sp0 + b) * Q + i)
                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
               }
 #pragma unroll
             for (int b = 0; b < UM_SPLIT_BATCH; ++b)
-              if (sp0 + b < p.splits)
+              if (sp0 + b < splits)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                   acc[u].x += v4[b][u].x;

@@ -50,3 +50,14 @@ def test_tcgen05_gemm_split_tail_wave(n, k):
     rows = [(0, 8), (5000, 5008), (n - 640, n - 632), (n - 8, n)]
     err = _run(n, k, 512, rows=rows, seed=4)
     assert err < TOL, err
+
+
+@pytest.mark.parametrize("m", [40, 64])
+def test_tcgen05_gemm_two_ctas_per_sm(m):
+    # 64-token tiles with at least as many tiles as SMs run two CTAs per SM
+    # (149 tiles of 128 rows, the last 56 rows): every row of the first two
+    # tiles, two tiles in the middle and the ragged last tile
+    n = 19000
+    rows = [(0, 256), (9472, 9728), (18944, n)]
+    err = _run(n, 1024, m, rows=rows, seed=6)
+    assert err < TOL, err
