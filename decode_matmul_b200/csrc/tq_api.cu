@@ -286,7 +286,7 @@ int umma_bn_for(int32_t m) { return m <= 64 ? 64 : (m <= 128 ? 128 : 256); }
 
 struct UmmaShape {
   int bn, row_tiles, tok_tiles, splits;
-  bool pair;  // 64-token tiles, two CTAs per SM (tq::UmmaSmem)
+  bool pair;  // 64- or 128-token tiles, two CTAs per SM (tq::UmmaSmem)
   size_t partial_bytes;
 };
 
@@ -301,7 +301,7 @@ UmmaShape umma_shape(int64_t n_total, int32_t k, int32_t m) {
   if (sp < 1) sp = 1;
   if (sp > blocks) sp = blocks;
   u.splits = sp;
-  u.pair = u.bn == 64 && tiles >= kSplitTarget;  // sp == 1 there
+  u.pair = u.bn <= 128 && tiles >= kSplitTarget;  // sp == 1 there
   u.partial_bytes = sp > 1 ? (size_t)tiles * sp * u.bn * tq::UM_BM * sizeof(float) : 0;
   return u;
 }
@@ -393,7 +393,7 @@ int umma_run(const uint8_t* const* codes, const uint16_t* const* scales, const i
   const int grid = u.row_tiles * u.tok_tiles * u.splits;
   switch (u.bn) {
     case 64: return u.pair ? umma_launch_t<64, true>(p, grid, stream) : umma_launch_t<64>(p, grid, stream);
-    case 128: return umma_launch_t<128>(p, grid, stream);
+    case 128: return u.pair ? umma_launch_t<128, true>(p, grid, stream) : umma_launch_t<128>(p, grid, stream);
     default: return umma_launch_t<256>(p, grid, stream);
   }
 }

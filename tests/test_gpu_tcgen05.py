@@ -52,9 +52,10 @@ def test_tcgen05_gemm_split_tail_wave(n, k):
     assert err < TOL, err
 
 
-@pytest.mark.parametrize("m", [40, 64])
+@pytest.mark.parametrize("m", [40, 64, 100, 128])
 def test_tcgen05_gemm_two_ctas_per_sm(m):
-    # 64-token tiles with at least as many tiles as SMs run two CTAs per SM
+    # 64- and 128-token tiles with at least as many tiles as SMs run two CTAs
+    # per SM
     # (149 tiles of 128 rows, the last 56 rows): every row of the first two
     # tiles, two tiles in the middle and the ragged last tile
     n = 19000
