@@ -180,11 +180,12 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // ---- shared-memory layout ---------------------------------------------------------
 
 // PAIR: two CTAs per SM (64- and 128-token tiles when there are at least as
-// many tiles as SMs): A in tensor memory, 6 stages at 64 tokens and 4 at 128,
-// 2 codebook views and 256 TMEM columns each, so that two fit one SM; the
+// many tiles as SMs): A in tensor memory, 4 stages, 4 codebook views at 64
+// tokens (2 at 128) and 256 TMEM columns each, so that two fit one SM; the
 // tiles then run in fewer waves and each SM has two independent stage
 // pipelines for the latency-bound loop (27B-class gate|up shape, 272 tiles:
-// 75.9 -> 56.0 us at 64 tokens, 87.0 -> 62.3 us at 128).  With fewer tiles
+// 75.9 -> 52.7 us at 64 tokens, 87.0 -> 62.3 us at 128; at 64 tokens 4
+// stages with 4 views measured 6% faster than 6 stages with 2).  With fewer tiles
 // (split k) the single-CTA form is faster; at 256-token tiles two CTAs do
 // not fit (their accumulators alone take all of TMEM).
 template <int BN, bool PAIR = false>
@@ -192,10 +193,10 @@ struct UmmaSmem {
   static_assert(!PAIR || BN <= 128, "two CTAs per SM at 64- and 128-token tiles only");
   // A in tensor memory at 64 and 256 tokens and in PAIR (see the file header)
   static constexpr bool TMEM_A = PAIR || BN != 128;
-  // stages: 12 at 64 tokens (6 in PAIR), 4 above; the codebook as 4 views
-  // (64 KB), 2 in PAIR
-  static constexpr int STAGES = PAIR ? (BN == 64 ? 6 : 4) : (BN == 64 ? 12 : 4);
-  static constexpr int LV = PAIR ? 1 : 2;
+  // stages: 12 at 64 tokens, 4 above and in PAIR; the codebook as 4 views
+  // (64 KB), 2 in PAIR at 128 tokens (4 stages of 18 KB leave no room for more)
+  static constexpr int STAGES = PAIR ? 4 : (BN == 64 ? 12 : 4);
+  static constexpr int LV = (PAIR && BN == 128) ? 1 : 2;
   // TMEM columns: the fp32 accumulator [0, BN), then (TMEM_A) 32 per stage
   static constexpr uint32_t A_COL0 = BN;
   static constexpr uint32_t TMEM_COLS = PAIR ? 256 : (TMEM_A ? 512 : BN);

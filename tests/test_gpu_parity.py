@@ -157,6 +157,23 @@ def test_gemm_two_row_tiles(tq, torch_cuda, m):
         assert err < TOL, (r0, err)
 
 
+@pytest.mark.parametrize("m", [32, 64])
+def test_gemm_repeatable_bits(tq, torch_cuda, m):
+    # tiles summed from several thread blocks' partials in a fixed order: the
+    # two-row-tile kernel at 32 tokens (27B-class down projection, every tile
+    # split over warps) and the tcgen05 kernel at 64 (the gate|up shape, two
+    # CTAs per SM; the down projection, split k) give the same bits every call
+    import torch
+    for n, k in [(5120, 17408), (34816, 5120)]:
+        hw = host_weight(8, 0, 2, n, k)
+        w = dev_weight(hw)
+        x = torch.from_numpy(np.random.default_rng(8).standard_normal((m, k)).astype(np.float16)).cuda()
+        ws = tq.workspace(tq.tq_gemm_workspace(n, k, m))
+        y0 = tq.tq_gemm(w, x, ws=ws)
+        for _ in range(2):
+            assert torch.equal(tq.tq_gemm(w, x, ws=ws), y0), (n, k, m)
+
+
 # ---- layer phases ------------------------------------------------------------------
 
 SMALL = tqsynth.StackShape("small", 2, 512, 1024, 512, 1536)
