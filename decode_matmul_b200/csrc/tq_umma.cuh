@@ -179,15 +179,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 // ---- shared-memory layout ---------------------------------------------------------
 
-// PAIR: two CTAs per SM (64- and 128-token tiles when there are at least as
-// many tiles as SMs): A in tensor memory, 4 stages, 4 codebook views at 64
+// PAIR: two CTAs per SM: A in tensor memory, 4 stages, 4 codebook views at 64
 // tokens (2 at 128) and 256 TMEM columns each, so that two fit one SM; the
-// tiles then run in fewer waves and each SM has two independent stage
-// pipelines for the latency-bound loop (27B-class gate|up shape, 272 tiles:
-// 75.9 -> 52.7 us at 64 tokens, 87.0 -> 62.3 us at 128; at 64 tokens 4
-// stages with 4 views measured 6% faster than 6 stages with 2).  With fewer tiles
-// (split k) the single-CTA form is faster; at 256-token tiles two CTAs do
-// not fit (their accumulators alone take all of TMEM).
+// tiles run in fewer waves and each SM has two independent stage pipelines
+// for the latency-bound loop (27B-class gate|up shape, 272 tiles: 75.9 ->
+// 52.7 us at 64 tokens, 87.0 -> 62.3 us at 128; at 64 tokens 4 stages with 4
+// views measured 6% faster than 6 stages with 2).  The host takes it for 64-
+// and 128-token tiles when there are at least as many tiles as SMs, and at 64
+// tokens also for split-k shapes whose splits (sized for two CTAs per SM)
+// keep at least 5 blocks each (27B-class down projection 46.8 -> 38.2 us);
+// shorter splits are faster in the single-CTA form.  At 256-token tiles two
+// CTAs do not fit (their accumulators alone take all of TMEM).
 template <int BN, bool PAIR = false>
 struct UmmaSmem {
   static_assert(!PAIR || BN <= 128, "two CTAs per SM at 64- and 128-token tiles only");
@@ -218,7 +220,7 @@ struct UmmaSmem {
 template <int BN, bool PAIR = false>
 __global__ void __launch_bounds__(UM_THREADS, PAIR ? 2 : 1) umma_kernel(const __grid_constant__ UmmaParams p) {
   using L = UmmaSmem<BN, PAIR>;
-  const int splits = PAIR ? 1 : p.splits;  // the host never splits k in PAIR
+  const int splits = p.splits;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -448,10 +450,11 @@ __global__ void __launch_bounds__(UM_THREADS, PAIR ? 2 : 1) umma_kernel(const __
           for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
           // the loads of up to UM_SPLIT_BATCH splits are all in flight before
           // the first add (the sum is latency-bound otherwise)
-          for (int sp0 = 0; sp0 < splits; sp0 += UM_SPLIT_BATCH) {
-            float4 v4[UM_SPLIT_BATCH][4];
+          constexpr int SB = PAIR ? 2 : UM_SPLIT_BATCH;  // fewer in flight in PAIR (register budget)
+          for (int sp0 = 0; sp0 < splits; sp0 += SB) {
+            float4 v4[SB][4];
 #pragma unroll
-            for (int b = 0; b < UM_SPLIT_BATCH; ++b)
+            for (int b = 0; b < SB; ++b)
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 const int i = i0 + u * UM_DEC_THREADS;
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(UM_THREADS, PAIR ? 2 : 1) umma_kernel(const __
                                                          : make_float4(0.f, 0.f, 0.f, 0.f);
               }
 #pragma unroll
-            for (int b = 0; b < UM_SPLIT_BATCH; ++b)
+            for (int b = 0; b < SB; ++b)
               if (sp0 + b < splits)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {

@@ -62,3 +62,10 @@ def test_tcgen05_gemm_two_ctas_per_sm(m):
     rows = [(0, 256), (9472, 9728), (18944, n)]
     err = _run(n, 1024, m, rows=rows, seed=6)
     assert err < TOL, err
+
+
+def test_tcgen05_gemm_two_ctas_per_sm_split_k():
+    # 40 row tiles at 48 tokens: k = 17408 split 7 ways (about 10 blocks each)
+    # for two CTAs per SM; rows of the first, a middle and the last tile
+    err = _run(5120, 17408, 48, rows=[(0, 128), (2560, 2688), (4992, 5120)], seed=7)
+    assert err < TOL, err
