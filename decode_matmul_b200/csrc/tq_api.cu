@@ -266,7 +266,7 @@ void dmma_single(DmmaParams& p, const tq_weight_t* w) {
 // ---- tcgen05 GEMM configuration -------------------------------------------------
 
 constexpr int kUmmaMinM = 33;  // from this many tokens on the decoded GEMM uses tcgen05 (measured crossover)
-constexpr int kSplitTarget = 148;    // split k until about one CTA per SM (B200 SM count)
+constexpr int kSplitTarget = 148;    // split k until about one CTA per SM (B200 SM count; two in PAIR)
 constexpr int kStatusOff = (int)kCounterBytes - 4;  // error word: last 4 bytes of the counter region
 static_assert(kStatusOff == TQ_STATUS_OFFSET, "the status word offset is part of the interface");
 
@@ -505,7 +505,7 @@ int run_phase(const tq_layer_t* L, int phase, const uint16_t* x, int32_t m, uint
     return dmma_run(p, true, ws, ws_bytes, num_sms, stream);
   }
   // m > 1: RHT to fp16 in the workspace tail, then the tcgen05 GEMM (m >= 33)
-  // or the small-batch kernel in chunks of up to 64 tokens.
+  // or the small-batch kernel in chunks of up to 32 tokens.
   const size_t dm_bytes = matmul_ws_bytes(n_total, k, m);
   uint16_t* xr = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + dm_bytes);
   int32_t rows[3];

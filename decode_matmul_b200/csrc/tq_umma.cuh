@@ -28,7 +28,8 @@
 //     leaves room for 12 stages of 10 KB (6 stages of 26 KB with A in shared
 //     memory were 15% faster than 4 on the 27B-class gate|up shape at 32
 //     tokens, 12 in TMEM another 4-5% at 64 tokens);
-//   * at 128 tokens, in shared memory (the K-major 128B-swizzled tile).
+//   * at 128 tokens, in shared memory (the K-major 128B-swizzled tile),
+//     except in the two-CTA form (PAIR, below), which keeps it in TMEM.
 // Stages are handed over with mbarriers; every wait is bounded and, when it
 // runs out, the kernel records TQ_ERR_TIMEOUT in the status word and drains.
 #pragma once
