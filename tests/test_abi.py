@@ -130,6 +130,22 @@ def test_gemv_k_limit_and_new_entry_points_checks():
     assert L.tq_gemm_ex(ctypes.byref(w), 16, 64, 16, 16, 1 << 30, ctypes.byref(opt), None) == tq.TQ_ERR_VALUE
 
 
+def test_gemm_workspace_covers_split_partials():
+    # the tcgen05 kernel's split-k partial sums ([tiles][splits][BN][128]
+    # fp32) live in the workspace after the 64 KB counter region; the query
+    # must cover the largest split the launcher can choose: 148 CTAs, or 296
+    # (two per SM) at 64-token tiles, and never more splits than 256-weight
+    # blocks
+    for n, k, m in [(5120, 17408, 48), (8192, 5120, 64), (2560, 9728, 64), (1040, 1536, 64), (2560, 4096, 512),
+                    (6144, 2560, 512), (128, 512, 200)]:
+        bn = 64 if m <= 64 else (128 if m <= 128 else 256)
+        tiles = -(-n // 128) * -(-m // bn)
+        blocks = k // 256
+        splits = min(max(1, (296 if bn == 64 else 148) // tiles), blocks)
+        need = 64 * 1024 + tiles * splits * bn * 128 * 4
+        assert tq.tq_gemm_workspace(n, k, m) >= need, (n, k, m)
+
+
 def test_stack_phase_seed_matches_oracle():
     # both sides implement SplitMix64 from its published definition
     for s, l, p in [(0, 0, 0), (0, 35, 3), (12345, 7, 2), (2 ** 64 - 1, 63, 1)]:
